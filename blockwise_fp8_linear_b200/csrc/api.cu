@@ -1,0 +1,194 @@
+// api.cu -- the C ABI of libfp8bw (declared in include/fp8bw.h): argument checks,
+// per-device properties, and dispatch to the quantizer and GEMM launchers.
+#include <atomic>
+#include <initializer_list>
+#include <cstdint>
+#include <cuda_runtime.h>
+
+#include "fp8bw.h"
+#include "quant.cuh"
+
+namespace {
+
+constexpr int kMaxDevices = 64;
+std::atomic<int> g_sms[kMaxDevices];    // 0 = not queried yet, -1 = not sm_100
+std::atomic<int> g_major[kMaxDevices];
+
+// Makes the device that owns the buffers current for this thread and returns its
+// SM count, or -1 with *status set.  Every pointer must be device (or managed)
+// memory of one device: a host pointer would fault the kernel, so it is rejected
+// here (FP8BW_EINVAL).
+int device_sms(std::initializer_list<const void *> ptrs, int *status)
+{
+    int dev = -1;
+    for (const void *p : ptrs) {
+        if (!p)
+            continue;
+        cudaPointerAttributes at;
+        if (cudaPointerGetAttributes(&at, p) != cudaSuccess) {
+            cudaGetLastError();
+            *status = FP8BW_ECUDA;
+            return -1;
+        }
+        if (at.type != cudaMemoryTypeDevice && at.type != cudaMemoryTypeManaged) {
+            *status = FP8BW_EINVAL;
+            return -1;
+        }
+        if (dev >= 0 && at.device != dev) {
+            *status = FP8BW_EINVAL;
+            return -1;
+        }
+        dev = at.device;
+    }
+    int cur = -1;
+    if (cudaGetDevice(&cur) != cudaSuccess) {
+        *status = FP8BW_ECUDA;
+        return -1;
+    }
+    if (dev < 0)
+        dev = cur;
+    if (dev != cur && cudaSetDevice(dev) != cudaSuccess) {
+        *status = FP8BW_ECUDA;
+        return -1;
+    }
+    if (dev >= kMaxDevices) {
+        *status = FP8BW_ECUDA;
+        return -1;
+    }
+    int sms = g_sms[dev].load(std::memory_order_acquire);
+    if (sms == 0) {
+        int major = 0, count = 0;
+        if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
+            cudaDeviceGetAttribute(&count, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) {
+            *status = FP8BW_ECUDA;
+            return -1;
+        }
+        g_major[dev].store(major, std::memory_order_relaxed);
+        sms = (major == 10) ? count : -1;
+        g_sms[dev].store(sms, std::memory_order_release);
+    }
+    if (sms < 0) {
+        *status = FP8BW_EUNSUPPORTED;
+        return -1;
+    }
+    *status = FP8BW_OK;
+    return sms;
+}
+
+bool aligned16(const void *p)
+{
+    return (reinterpret_cast<uintptr_t>(p) & 15u) == 0;
+}
+
+bool dim_ok(int64_t d)
+{
+    return d > 0 && d <= FP8BW_MAX_DIM && (d % 128) == 0;
+}
+
+int from_cuda(cudaError_t e)
+{
+    return e == cudaSuccess ? FP8BW_OK : FP8BW_ECUDA;
+}
+
+} // namespace
+
+extern "C" {
+
+int fp8_quant_act(const void *x_bf16, int64_t M, int64_t K, uint8_t *q, float *s, void *stream)
+{
+    if (!x_bf16 || !q || !s)
+        return FP8BW_EINVAL;
+    if (!dim_ok(M) || !dim_ok(K))
+        return FP8BW_ESHAPE;
+    if (!aligned16(x_bf16) || !aligned16(q) || !aligned16(s))
+        return FP8BW_EALIGN;
+    int st;
+    const int sms = device_sms({x_bf16, q, s}, &st);
+    if (sms < 0)
+        return st;
+    return from_cuda(fp8bw::launch_quant_act(x_bf16, M, K, q, s,
+                                             static_cast<cudaStream_t>(stream), sms));
+}
+
+int fp8_quant_act_t(const void *x_bf16, int64_t M, int64_t K, uint8_t *qt, float *st_,
+                    void *stream)
+{
+    if (!x_bf16 || !qt || !st_)
+        return FP8BW_EINVAL;
+    if (!dim_ok(M) || !dim_ok(K))
+        return FP8BW_ESHAPE;
+    if (!aligned16(x_bf16) || !aligned16(qt) || !aligned16(st_))
+        return FP8BW_EALIGN;
+    int st;
+    if (device_sms({x_bf16, qt, st_}, &st) < 0)
+        return st;
+    return from_cuda(
+        fp8bw::launch_quant_act_t(x_bf16, M, K, qt, st_, static_cast<cudaStream_t>(stream)));
+}
+
+int fp8_quant_weight(const void *w_bf16, int64_t N, int64_t K, uint8_t *q, float *s,
+                     uint8_t *qt_or_null, void *stream)
+{
+    if (!w_bf16 || !q || !s)
+        return FP8BW_EINVAL;
+    if (!dim_ok(N) || !dim_ok(K))
+        return FP8BW_ESHAPE;
+    if (!aligned16(w_bf16) || !aligned16(q) || !aligned16(s) ||
+        (qt_or_null && !aligned16(qt_or_null)))
+        return FP8BW_EALIGN;
+    int st;
+    if (device_sms({w_bf16, q, s, qt_or_null}, &st) < 0)
+        return st;
+    return from_cuda(fp8bw::launch_quant_weight(w_bf16, N, K, q, s, qt_or_null,
+                                                static_cast<cudaStream_t>(stream)));
+}
+
+int fp8_gemm_blockwise(int mode, const uint8_t *a, const float *sa, const uint8_t *b,
+                       const float *sb, void *d_bf16, int64_t M, int64_t N, int64_t K,
+                       void *stream)
+{
+    if (mode < FP8BW_FPROP || mode > FP8BW_WGRAD || !a || !sa || !b || !sb || !d_bf16)
+        return FP8BW_EINVAL;
+    if (!dim_ok(M) || !dim_ok(N) || !dim_ok(K))
+        return FP8BW_ESHAPE;
+    if (!aligned16(a) || !aligned16(sa) || !aligned16(b) || !aligned16(sb) || !aligned16(d_bf16))
+        return FP8BW_EALIGN;
+    int st;
+    const int sms = device_sms({a, sa, b, sb, d_bf16}, &st);
+    if (sms < 0)
+        return st;
+    return from_cuda(fp8bw::launch_gemm(mode, a, sa, b, sb, d_bf16, M, N, K,
+                                        static_cast<cudaStream_t>(stream), sms));
+}
+
+const char *fp8bw_status_string(int status)
+{
+    switch (status) {
+    case FP8BW_OK: return "FP8BW_OK";
+    case FP8BW_EINVAL: return "FP8BW_EINVAL: null pointer or invalid mode";
+    case FP8BW_EALIGN: return "FP8BW_EALIGN: pointer not 16-byte aligned";
+    case FP8BW_ESHAPE: return "FP8BW_ESHAPE: size not a positive multiple of 128 (or too large)";
+    case FP8BW_ECUDA: return "FP8BW_ECUDA: CUDA runtime error";
+    case FP8BW_ETIMEOUT: return "FP8BW_ETIMEOUT: a bounded in-kernel wait ran out";
+    case FP8BW_EUNSUPPORTED: return "FP8BW_EUNSUPPORTED: device is not sm_100";
+    default: return "unknown fp8bw status";
+    }
+}
+
+int fp8bw_last_device_error(void *stream)
+{
+    int st;
+    if (device_sms({}, &st) < 0)
+        return st;
+    int v = 0;
+    if (fp8bw::read_and_clear_device_error(static_cast<cudaStream_t>(stream), &v) != cudaSuccess)
+        return FP8BW_ECUDA;
+    return v ? FP8BW_ETIMEOUT : FP8BW_OK;
+}
+
+const char *fp8bw_version(void)
+{
+    return "fp8bw 0.1 sm_100a";
+}
+
+} // extern "C"

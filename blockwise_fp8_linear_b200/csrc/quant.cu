@@ -1,0 +1,302 @@
+// quant.cu -- E4M3 quantizers for the blockwise-FP8 linear layer (sm_100a).
+//
+// Three layouts (Puro-2B part 3/7, section 3.2): 1x128 groups along the reduction
+// dimension for activations / activation gradients, the same groups taken along the
+// token dimension for wgrad, and 128x128 blocks for weights.  Each group's scale is
+// amax/448 in FP32 (one IEEE division); each value is divided by the scale with the
+// quotient rounded to FP32, then rounded to nearest-even onto E4M3 with saturation
+// at +-448 (cvt.rn.satfinite).  An all-zero group gets scale 0 and codes 0x00.
+//
+// All three kernels are HBM-bound streaming kernels: 2 bytes read and 1 + 4/128
+// bytes written per element.
+#include <cstdint>
+#include <cuda_runtime.h>
+
+#include "quant.cuh"
+
+namespace fp8bw {
+
+// Two FP32 values -> two E4M3 codes (RNE, saturating); `lo` lands in the low byte.
+__device__ __forceinline__ uint32_t cvt_e4m3x2(float lo, float hi)
+{
+    uint16_t r;
+    asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(r) : "f"(hi), "f"(lo));
+    return r;
+}
+
+// Per-group division x / s, correctly rounded to binary32.
+//
+// Fast path (s in [2^-90, 2^90]): one correctly rounded reciprocal r = RN(1/s) per
+// group, then per value q0 = RN(x*r), e = x - q0*s (exact by FMA) and
+// q = RN(q0 + e*r).  By Markstein's theorem (P. Markstein, "Computation of elementary
+// functions on the IBM RISC System/6000 processor", IBM J. Res. Dev. 34(1), 1990;
+// also Muller et al., Handbook of Floating-Point Arithmetic, ch. 4) this is the
+// correctly rounded quotient whenever no intermediate underflows; quotients small
+// enough for that to matter lie far below half the smallest E4M3 subnormal (2^-10),
+// where only the sign survives, and the sign is restored from x.  Outside that
+// range of s the group falls back to the compiler's IEEE division.  The test suite
+// checks the fast path against IEEE division for every (BF16 amax, BF16 x) pair.
+struct GroupDiv {
+    float s, r;
+    bool fast;
+    __device__ __forceinline__ explicit GroupDiv(float scale) : s(scale)
+    {
+        fast = scale >= 0x1p-90f && scale <= 0x1p90f;
+        r = fast ? __frcp_rn(scale) : 0.0f;
+    }
+    __device__ __forceinline__ float operator()(float x) const
+    {
+        if (fast) {
+            float q0 = __fmul_rn(x, r);
+            float e = __fmaf_rn(-q0, s, x);
+            float q = __fmaf_rn(e, r, q0);
+            return copysignf(q, x);
+        }
+        return __fdiv_rn(x, s);
+    }
+};
+
+__device__ __forceinline__ float bf16lo(uint32_t w) { return __uint_as_float(w << 16); }
+__device__ __forceinline__ float bf16hi(uint32_t w) { return __uint_as_float(w & 0xFFFF0000u); }
+
+// |bf16| max over two packed words, as packed unsigned 16-bit halves (for
+// non-negative BF16 values the integer order is the numeric order).
+__device__ __forceinline__ uint32_t absmax2(uint32_t a, uint32_t b)
+{
+    return __vmaxu2(a & 0x7FFF7FFFu, b & 0x7FFF7FFFu);
+}
+
+__device__ __forceinline__ float halves_max_to_float(uint32_t m2)
+{
+    uint32_t m = max(m2 & 0xFFFFu, m2 >> 16);
+    return __uint_as_float(m << 16);
+}
+
+// Eight BF16 values (one uint4) -> eight E4M3 codes (one uint2).
+__device__ __forceinline__ uint2 quant8(uint4 v, const GroupDiv &div)
+{
+    uint2 o;
+    o.x = cvt_e4m3x2(div(bf16lo(v.x)), div(bf16hi(v.x))) |
+          (cvt_e4m3x2(div(bf16lo(v.y)), div(bf16hi(v.y))) << 16);
+    o.y = cvt_e4m3x2(div(bf16lo(v.z)), div(bf16hi(v.z))) |
+          (cvt_e4m3x2(div(bf16lo(v.w)), div(bf16hi(v.w))) << 16);
+    return o;
+}
+
+// ------------------------------------------------------------ fp8_quant_act
+
+// A warp quantizes two groups at a time: half-warp h takes group (kb, m + h); each
+// lane holds 8 consecutive values (16 bytes).  Groups are enumerated g = kb*M + m
+// so the scale writes of neighbouring warps are contiguous.
+constexpr int QA_THREADS = 256;
+constexpr int QA_UNROLL = 4;
+
+__global__ void __launch_bounds__(QA_THREADS)
+quant_act_kernel(const uint4 *__restrict__ x, int64_t M, int64_t K, uint2 *__restrict__ q,
+                 float *__restrict__ s)
+{
+    const int64_t npairs = M * (K / 128) / 2;
+    const int64_t warp = (int64_t(blockIdx.x) * QA_THREADS + threadIdx.x) >> 5;
+    const int64_t nwarps = (int64_t(gridDim.x) * QA_THREADS) >> 5;
+    const int lane = threadIdx.x & 31;
+    const int half = lane >> 4, sub = lane & 15;
+
+    for (int64_t p0 = warp; p0 < npairs; p0 += nwarps * QA_UNROLL) {
+        uint4 v[QA_UNROLL];
+        int64_t off[QA_UNROLL];
+#pragma unroll
+        for (int u = 0; u < QA_UNROLL; ++u) {
+            int64_t p = p0 + int64_t(u) * nwarps;
+            off[u] = -1;
+            if (p < npairs) {
+                int64_t g = 2 * p + half;
+                int64_t kb = g / M, m = g - kb * M;
+                off[u] = (m * K + kb * 128) / 8 + sub;  // in units of 8 elements
+                v[u] = __ldg(x + off[u]);
+            }
+        }
+#pragma unroll
+        for (int u = 0; u < QA_UNROLL; ++u) {
+            int64_t p = p0 + int64_t(u) * nwarps;
+            if (p >= npairs)  // uniform across the warp
+                break;
+            uint32_t m2 = __vmaxu2(absmax2(v[u].x, v[u].y), absmax2(v[u].z, v[u].w));
+#pragma unroll
+            for (int o = 8; o >= 1; o >>= 1)
+                m2 = __vmaxu2(m2, __shfl_xor_sync(0xffffffffu, m2, o));
+            float amax = halves_max_to_float(m2);
+            float sc = __fdiv_rn(amax, 448.0f);
+            uint2 codes = make_uint2(0u, 0u);
+            if (amax != 0.0f)
+                codes = quant8(v[u], GroupDiv(sc));
+            q[off[u]] = codes;
+            if (sub == 0)
+                s[2 * p + half] = sc;
+        }
+    }
+}
+
+// ---------------------------------------------------------- fp8_quant_act_t
+
+// Block tile: 128 rows (one token block mb) x 64 columns.  Warp w holds rows
+// 16w .. 16w+15; lane l holds columns 2l and 2l+1 of every one of those rows.
+// Column absmax: per lane over its 16 rows, then across the 8 warps in shared
+// memory.  Each lane then owns 16 consecutive tokens of two columns, which are 16
+// contiguous bytes of the transposed output: one 16-byte store per column.
+constexpr int QT_THREADS = 256;
+
+__global__ void __launch_bounds__(QT_THREADS)
+quant_act_t_kernel(const uint32_t *__restrict__ x, int64_t M, int64_t K,
+                   uint8_t *__restrict__ qt, float *__restrict__ st)
+{
+    __shared__ uint32_t red[8][32];
+    const int w = threadIdx.x >> 5, l = threadIdx.x & 31;
+    const int64_t k0 = int64_t(blockIdx.x) * 64;
+    const int64_t mb = blockIdx.y;
+    const int64_t row0 = mb * 128 + 16 * w;
+
+    uint32_t v[16];
+#pragma unroll
+    for (int r = 0; r < 16; ++r)
+        v[r] = __ldg(x + ((row0 + r) * K + k0) / 2 + l);
+    uint32_t m2 = 0;
+#pragma unroll
+    for (int r = 0; r < 16; r += 2)
+        m2 = __vmaxu2(m2, absmax2(v[r], v[r + 1]));
+    red[w][l] = m2;
+    __syncthreads();
+#pragma unroll
+    for (int i = 0; i < 8; ++i)
+        m2 = __vmaxu2(m2, red[i][l]);
+
+    const float amax_lo = __uint_as_float((m2 & 0xFFFFu) << 16);
+    const float amax_hi = __uint_as_float(m2 & 0xFFFF0000u);
+    const float s_lo = __fdiv_rn(amax_lo, 448.0f);
+    const float s_hi = __fdiv_rn(amax_hi, 448.0f);
+
+    uint32_t clo[4] = {0u, 0u, 0u, 0u}, chi[4] = {0u, 0u, 0u, 0u};
+    if (amax_lo != 0.0f) {
+        GroupDiv d(s_lo);
+#pragma unroll
+        for (int r = 0; r < 16; r += 2)
+            clo[r / 4] |= cvt_e4m3x2(d(bf16lo(v[r])), d(bf16lo(v[r + 1]))) << (16 * ((r / 2) & 1));
+    }
+    if (amax_hi != 0.0f) {
+        GroupDiv d(s_hi);
+#pragma unroll
+        for (int r = 0; r < 16; r += 2)
+            chi[r / 4] |= cvt_e4m3x2(d(bf16hi(v[r])), d(bf16hi(v[r + 1]))) << (16 * ((r / 2) & 1));
+    }
+    const int64_t col = k0 + 2 * l;
+    *reinterpret_cast<uint4 *>(qt + col * M + row0) = make_uint4(clo[0], clo[1], clo[2], clo[3]);
+    *reinterpret_cast<uint4 *>(qt + (col + 1) * M + row0) = make_uint4(chi[0], chi[1], chi[2], chi[3]);
+    if (w == 0)
+        *reinterpret_cast<float2 *>(st + mb * K + col) = make_float2(s_lo, s_hi);
+}
+
+// --------------------------------------------------------- fp8_quant_weight
+
+// One block per 128x128 weight block.  Thread t covers, in each of 8 passes, row
+// pass*16 + t/16 and columns (t%16)*8 .. +7.
+constexpr int QW_THREADS = 256;
+
+__global__ void __launch_bounds__(QW_THREADS)
+quant_weight_kernel(const uint4 *__restrict__ w, int64_t N, int64_t K, uint2 *__restrict__ q,
+                    float *__restrict__ s, uint8_t *__restrict__ qt)
+{
+    __shared__ uint32_t red[8];
+    __shared__ uint8_t tile[128][144];  // codes, for the optional transposed copy
+    const int t = threadIdx.x;
+    const int64_t kb = blockIdx.x, nb = blockIdx.y;
+    const int rsub = t >> 4, csub = (t & 15) * 8;
+
+    uint4 v[8];
+#pragma unroll
+    for (int p = 0; p < 8; ++p) {
+        int64_t n = nb * 128 + p * 16 + rsub;
+        v[p] = __ldg(w + (n * K + kb * 128 + csub) / 8);
+    }
+    uint32_t m2 = 0;
+#pragma unroll
+    for (int p = 0; p < 8; ++p)
+        m2 = __vmaxu2(m2, __vmaxu2(absmax2(v[p].x, v[p].y), absmax2(v[p].z, v[p].w)));
+#pragma unroll
+    for (int o = 16; o >= 1; o >>= 1)
+        m2 = __vmaxu2(m2, __shfl_xor_sync(0xffffffffu, m2, o));
+    if ((t & 31) == 0)
+        red[t >> 5] = m2;
+    __syncthreads();
+#pragma unroll
+    for (int i = 0; i < 8; ++i)
+        m2 = __vmaxu2(m2, red[i]);
+    const float amax = halves_max_to_float(m2);
+    const float sc = __fdiv_rn(amax, 448.0f);
+    const GroupDiv div(sc);
+
+#pragma unroll
+    for (int p = 0; p < 8; ++p) {
+        int64_t n = nb * 128 + p * 16 + rsub;
+        uint2 c = make_uint2(0u, 0u);
+        if (amax != 0.0f)
+            c = quant8(v[p], div);
+        q[(n * K + kb * 128 + csub) / 8] = c;
+        if (qt)
+            *reinterpret_cast<uint2 *>(&tile[p * 16 + rsub][csub]) = c;
+    }
+    if (t == 0)
+        s[nb * (K / 128) + kb] = sc;
+    if (qt) {
+        __syncthreads();
+        // qt[k][n]: thread t writes column k = t/2 of the block, 64 rows starting at
+        // (t%2)*64, as four 16-byte stores.
+        const int kk = t >> 1, n0 = (t & 1) * 64;
+        uint8_t *dst = qt + (kb * 128 + kk) * N + nb * 128 + n0;
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+            uint32_t wv[4];
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+                const int r = n0 + c * 16 + j * 4;
+                wv[j] = uint32_t(tile[r][kk]) | (uint32_t(tile[r + 1][kk]) << 8) |
+                        (uint32_t(tile[r + 2][kk]) << 16) | (uint32_t(tile[r + 3][kk]) << 24);
+            }
+            *reinterpret_cast<uint4 *>(dst + c * 16) = make_uint4(wv[0], wv[1], wv[2], wv[3]);
+        }
+    }
+}
+
+// ------------------------------------------------------------------ launchers
+
+cudaError_t launch_quant_act(const void *x, int64_t M, int64_t K, uint8_t *q, float *s,
+                             cudaStream_t stream, int num_sms)
+{
+    const int64_t npairs = M * (K / 128) / 2;
+    const int64_t warps_needed = (npairs + QA_UNROLL - 1) / QA_UNROLL;
+    int64_t blocks = (warps_needed + (QA_THREADS / 32) - 1) / (QA_THREADS / 32);
+    const int64_t cap = int64_t(num_sms) * 8;
+    if (blocks > cap)
+        blocks = cap;
+    quant_act_kernel<<<dim3(unsigned(blocks)), QA_THREADS, 0, stream>>>(
+        static_cast<const uint4 *>(x), M, K, reinterpret_cast<uint2 *>(q), s);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_quant_act_t(const void *x, int64_t M, int64_t K, uint8_t *qt, float *st,
+                               cudaStream_t stream)
+{
+    dim3 grid(unsigned(K / 64), unsigned(M / 128));
+    quant_act_t_kernel<<<grid, QT_THREADS, 0, stream>>>(static_cast<const uint32_t *>(x), M, K,
+                                                       qt, st);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_quant_weight(const void *w, int64_t N, int64_t K, uint8_t *q, float *s,
+                                uint8_t *qt, cudaStream_t stream)
+{
+    dim3 grid(unsigned(K / 128), unsigned(N / 128));
+    quant_weight_kernel<<<grid, QW_THREADS, 0, stream>>>(
+        static_cast<const uint4 *>(w), N, K, reinterpret_cast<uint2 *>(q), s, qt);
+    return cudaGetLastError();
+}
+
+} // namespace fp8bw

@@ -1,0 +1,25 @@
+// quant.cuh -- launchers of the quantizer kernels (internal to libfp8bw).
+#pragma once
+
+#include <cstdint>
+#include <cuda_runtime.h>
+
+namespace fp8bw {
+
+cudaError_t launch_quant_act(const void *x, int64_t M, int64_t K, uint8_t *q, float *s,
+                             cudaStream_t stream, int num_sms);
+cudaError_t launch_quant_act_t(const void *x, int64_t M, int64_t K, uint8_t *qt, float *st,
+                               cudaStream_t stream);
+cudaError_t launch_quant_weight(const void *w, int64_t N, int64_t K, uint8_t *q, float *s,
+                                uint8_t *qt, cudaStream_t stream);
+
+// GEMM: D[M][N] bf16 from FP8 operands with blockwise scales (mode 0/1/2 =
+// fprop/dgrad/wgrad).  Arguments already validated.
+cudaError_t launch_gemm(int mode, const uint8_t *a, const float *sa, const uint8_t *b,
+                        const float *sb, void *d, int64_t M, int64_t N, int64_t K,
+                        cudaStream_t stream, int num_sms);
+
+// Per-device error word written by bounded in-kernel waits.
+cudaError_t read_and_clear_device_error(cudaStream_t stream, int *value);
+
+} // namespace fp8bw

@@ -1,0 +1,137 @@
+/*
+ * fp8bw.h -- C ABI of the blockwise-FP8 Transformer linear layer for NVIDIA B200
+ * (sm_100a).
+ *
+ * The operations follow Puro-2B ("Poor Lab's Qwen2-1.5B Trained on RTX 5090 within
+ * $5090", arXiv HTML part 3/7), section 3.2 "FP8 Mixed-Precision Training":
+ * Transformer linear layers quantize their BF16 inputs and weights to E4M3
+ * immediately before each GEMM, with one scale per 128 consecutive values along the
+ * GEMM reduction dimension for activations and activation gradients and one scale
+ * per 128x128 block for weights; fprop, dgrad and wgrad all run in FP8 and the layer
+ * hands a BF16 result back to the model.  Each block scale is the block's absolute
+ * maximum divided by 448 (the largest finite E4M3 magnitude) in FP32, and values are
+ * divided by it and rounded to nearest-even onto E4M3, saturating at +-448 (the
+ * fine-grained recipe section 3.2 says it follows, DeepSeek-V3).
+ *
+ * Conventions for every entry point
+ *   Pointers     Device pointers on the calling thread's current CUDA device, unless
+ *                stated otherwise.  The caller allocates and owns every buffer; the
+ *                library never frees caller memory and keeps no pointer after the
+ *                call returns.
+ *   Layouts      Row-major [rows][cols].  BF16 tensors are IEEE bfloat16.  FP8 codes
+ *                are E4M3 ("E4M3FN": bias 7, no infinities, NaN = S.1111.111).
+ *                1x128 scale tensors are reduction-block-major, s[kb][row], so one
+ *                tile's scales for one reduction block are contiguous.
+ *   Sizes        Every dimension must be a positive multiple of 128 and at most
+ *                FP8BW_MAX_DIM (else FP8BW_ESHAPE).
+ *   Alignment    Every pointer must be 16-byte aligned (else FP8BW_EALIGN).
+ *   Streams      `stream` is a cudaStream_t (NULL = legacy default stream).  Work is
+ *                enqueued asynchronously; no call synchronizes the stream.  Calls on
+ *                distinct streams may run concurrently from different threads.
+ *   Errors       Every call returns an fp8bw_status and never aborts or throws.
+ *                Argument errors are reported before anything is launched.  A failed
+ *                launch returns FP8BW_ECUDA.  The GEMM bounds every wait inside the
+ *                kernel; a wait that runs out sets a per-device error word that
+ *                fp8bw_last_device_error() reads.
+ *   Inputs       Finite BF16 values.  Non-finite inputs give unspecified codes but
+ *                never fault.
+ *   Memory       The library allocates no device memory: the per-device error word
+ *                is a static device variable and TMA descriptors are passed by value.
+ */
+#ifndef FP8BW_H
+#define FP8BW_H
+
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    FP8BW_OK = 0,
+    FP8BW_EINVAL = 1,      /* null pointer or bad mode */
+    FP8BW_EALIGN = 2,      /* a pointer is not 16-byte aligned */
+    FP8BW_ESHAPE = 3,      /* a size is not a positive multiple of 128, or too large */
+    FP8BW_ECUDA = 4,       /* a CUDA runtime call or kernel launch failed */
+    FP8BW_ETIMEOUT = 5,    /* a bounded in-kernel wait ran out (from fp8bw_last_device_error) */
+    FP8BW_EUNSUPPORTED = 6 /* the current device is not sm_100 */
+} fp8bw_status;
+
+typedef enum { FP8BW_FPROP = 0, FP8BW_DGRAD = 1, FP8BW_WGRAD = 2 } fp8bw_mode;
+
+#define FP8BW_MAX_DIM (1 << 20)
+
+/*
+ * fp8_quant_act -- 1x128 groups along the reduction dimension (section 3.2:
+ * "activations and activation gradients use one-dimensional groups of 128
+ * consecutive values along the GEMM reduction dimension").
+ *   x  [M][K] BF16 in      q [M][K] E4M3 codes out      s [K/128][M] FP32 out
+ * For each row m and block kb: amax = max |x[m][kb*128 .. kb*128+127]|,
+ * s[kb][m] = amax / 448 (binary32 division), q = e4m3_rne_sat(x / s) with the
+ * quotient rounded to binary32 first.  An all-zero group gets s = 0 and codes 0x00.
+ * Used for X before fprop (K = in_features) and dY before dgrad (K = out_features).
+ */
+int fp8_quant_act(const void *x_bf16, int64_t M, int64_t K, uint8_t *q, float *s,
+                  void *stream);
+
+/*
+ * fp8_quant_act_t -- the same groups taken along M (the token dimension), the
+ * grouping wgrad needs because its reduction runs over tokens (section 3.2: wgrad
+ * runs in FP8 on the layer's inputs and output gradients).
+ *   x  [M][K] BF16 in      qt [K][M] E4M3 codes out (transposed)      st [M/128][K] FP32 out
+ * For each column k and block mb: the group is x[mb*128 .. mb*128+127][k];
+ * st[mb][k] is its scale and qt[k][mb*128 + i] its codes.  Quantized from the BF16
+ * tensor, not from the row-wise FP8 copy.
+ */
+int fp8_quant_act_t(const void *x_bf16, int64_t M, int64_t K, uint8_t *qt, float *st,
+                    void *stream);
+
+/*
+ * fp8_quant_weight -- 128x128 blocks (section 3.2: "weights use two-dimensional
+ * 128x128 blocks").
+ *   w  [N][K] BF16 in      q [N][K] E4M3 out      s [N/128][K/128] FP32 out
+ *   qt_or_null: if not NULL, also writes qt [K][N] = q transposed (same codes; a
+ *   128x128 block keeps its one scale under transposition).
+ */
+int fp8_quant_weight(const void *w_bf16, int64_t N, int64_t K, uint8_t *q, float *s,
+                     uint8_t *qt_or_null, void *stream);
+
+/*
+ * fp8_gemm_blockwise -- D[M][N] (BF16) = sum over a reduction of length K, with the
+ * reduction cut into 128-long blocks kb.  For each kb the FP8 partial product
+ * sum_{k in kb} qa*qb is accumulated in FP32 by the tensor cores and then promoted
+ * into an FP32 running sum multiplied by (a-scale x b-scale) of that block; the sum
+ * is rounded to BF16 (nearest-even) at the end.  Section 3.2: "their Fprop, Dgrad,
+ * and Wgrad GEMMs all use the FP8 path", with a BF16 output for the model.
+ *
+ *   FPROP  Y  = X . W^T   a = Qx  [M][K], sa = [K/128][M]   (from fp8_quant_act(X))
+ *                         b = Qw  [N][K], sb = [N/128][K/128] (from fp8_quant_weight(W))
+ *                         M = tokens, K = in_features, N = out_features
+ *   DGRAD  dX = dY . W    a = Qdy [M][K], sa = [K/128][M]   (from fp8_quant_act(dY))
+ *                         b = Qw  [K][N], sb = [K/128][N/128] (the weight exactly as
+ *                         fp8_quant_weight produced it, [out][in]; read transposed)
+ *                         M = tokens, K = out_features, N = in_features
+ *   WGRAD  dW = dY^T . X  a = Qdy^T [M][K], sa = [K/128][M] (from fp8_quant_act_t(dY))
+ *                         b = Qx^T  [N][K], sb = [K/128][N] (from fp8_quant_act_t(X))
+ *                         M = out_features, K = tokens, N = in_features
+ * d_bf16 [M][N] is written, never read.
+ */
+int fp8_gemm_blockwise(int mode, const uint8_t *a, const float *sa, const uint8_t *b,
+                       const float *sb, void *d_bf16, int64_t M, int64_t N, int64_t K,
+                       void *stream);
+
+/* Human-readable name of a status code (static string). */
+const char *fp8bw_status_string(int status);
+
+/* Synchronizes `stream`, then reads and clears the current device's error word:
+ * FP8BW_OK, or FP8BW_ETIMEOUT if a bounded in-kernel wait ran out since the last
+ * call (the GEMM whose wait ran out returned early and its output is undefined). */
+int fp8bw_last_device_error(void *stream);
+
+/* Library version, e.g. "fp8bw 0.1 sm_100a". */
+const char *fp8bw_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* FP8BW_H */

@@ -1,0 +1,151 @@
+"""GPU parity of fp8_gemm_blockwise (fprop / dgrad / wgrad) against the CPU oracle's
+FP64 GEMM over the oracle's own quantized operands.
+
+The GPU GEMM consumes the GPU quantizers' output; those are checked bit-exact
+against the oracle's first, so both sides see the same FP8 bytes and scales."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from blockwise_fp8_linear_b200 import (DGRAD, FPROP, WGRAD, fp8_gemm_blockwise, fp8_quant_act,
+                                       fp8_quant_act_t, fp8_quant_weight, synth)
+from tests._gpu import bf16_dev_to_f64, check_gemm, to_dev_bf16
+
+pytestmark = pytest.mark.gpu
+
+
+def _same(gpu: torch.Tensor, ref: np.ndarray):
+    g = gpu.cpu().numpy()
+    if ref.dtype == np.float32:
+        assert np.array_equal(g.view(np.uint32), ref.view(np.uint32))
+    else:
+        assert np.array_equal(g, ref)
+
+
+def _layer(T, Din, Dout, seed, outliers=True):
+    X = synth.normal_bf16(T, Din, 1.0, seed=synth.seed_for(seed, 0), outliers=outliers)
+    W = synth.normal_bf16(Dout, Din, 0.02, seed=synth.seed_for(seed, 1))
+    dY = synth.normal_bf16(T, Dout, 1e-3, seed=synth.seed_for(seed, 2))
+    return X, W, dY
+
+
+def _rows(M, n):
+    """A deterministic spread of rows touching every 128-row tile (first and last
+    rows of tiles included)."""
+    if M <= n:
+        return np.arange(M)
+    rng = np.random.default_rng(M)
+    base = np.concatenate([np.arange(0, M, 128), np.arange(127, M, 128)])
+    extra = rng.choice(M, max(0, n - base.size), replace=False)
+    return np.unique(np.concatenate([base, extra]))[:max(n, base.size)]
+
+
+def _run_mode(mode, X, W, dY, rows=None):
+    """Quantize on both sides, check the bytes, run the GEMM, return (y, y_ref, asum)."""
+    T, Din = X.shape
+    Dout = W.shape[0]
+    if mode == FPROP:
+        a_d, sa_d = fp8_quant_act(to_dev_bf16(X))
+        b_d, sb_d, _ = fp8_quant_weight(to_dev_bf16(W))
+        a, sa = oracle.quant_act(X)
+        b, sb, _ = oracle.quant_weight(W)
+        M, N, K = T, Dout, Din
+    elif mode == DGRAD:
+        a_d, sa_d = fp8_quant_act(to_dev_bf16(dY))
+        b_d, sb_d, _ = fp8_quant_weight(to_dev_bf16(W))
+        a, sa = oracle.quant_act(dY)
+        b, sb, _ = oracle.quant_weight(W)
+        M, N, K = T, Din, Dout
+    else:
+        a_d, sa_d = fp8_quant_act_t(to_dev_bf16(dY))
+        b_d, sb_d = fp8_quant_act_t(to_dev_bf16(X))
+        a, sa = oracle.quant_act_t(dY)
+        b, sb = oracle.quant_act_t(X)
+        M, N, K = Dout, Din, T
+    for g, r in ((a_d, a), (sa_d, sa), (b_d, b), (sb_d, sb)):
+        _same(g, r)
+    y = bf16_dev_to_f64(fp8_gemm_blockwise(mode, a_d, sa_d, b_d, sb_d, M, N, K))
+    y_ref, asum = oracle.gemm(mode, a, sa, b, sb, M, N, K, rows=rows)
+    if rows is not None:
+        y = y[rows]
+    return y, y_ref, asum
+
+
+@pytest.mark.parametrize("mode", [FPROP, DGRAD, WGRAD])
+@pytest.mark.parametrize("T,Din,Dout", [
+    (128, 1024, 1024),   # the single-fprop workload's shape (one row-tile)
+    (384, 640, 896),     # N not a multiple of 256: the 128-wide tile path, ragged grid
+    (256, 1152, 768),    # 3 tiles of 256 columns, odd number of reduction blocks
+    (1024, 256, 2048),   # more column tiles, short reduction
+])
+def test_gemm_small_full(mode, T, Din, Dout):
+    X, W, dY = _layer(T, Din, Dout, seed=T + Din + Dout + mode)
+    y, y_ref, asum = _run_mode(mode, X, W, dY)
+    check_gemm(y, y_ref, asum, f"mode {mode} {T}x{Din}x{Dout}")
+
+
+def test_gemm_single_fprop_workload():
+    """X[128x1024] ~ N(0,1), W[1024x1024] ~ N(0,0.02), seed 0: Y = X W^T, checked
+    on every output."""
+    X = synth.normal_bf16(128, 1024, 1.0, seed=synth.seed_for(0, 0))
+    W = synth.normal_bf16(1024, 1024, 0.02, seed=synth.seed_for(0, 1))
+    y, y_ref, asum = _run_mode(FPROP, X, W, None)
+    check_gemm(y, y_ref, asum, "single fprop")
+
+
+@pytest.mark.parametrize("mode", [FPROP, DGRAD, WGRAD])
+def test_gemm_many_tiles_per_cta(mode):
+    """More tiles than SMs, so each persistent CTA walks several tiles and both TMEM
+    buffers wrap many times; rows sampled across every row-tile."""
+    T, Din, Dout = 2048, 1024, 3072
+    X, W, dY = _layer(T, Din, Dout, seed=77 + mode)
+    M = {FPROP: T, DGRAD: T, WGRAD: Dout}[mode]
+    rows = _rows(M, 64)
+    y, y_ref, asum = _run_mode(mode, X, W, dY, rows=rows)
+    check_gemm(y, y_ref, asum, f"mode {mode} many tiles")
+
+
+# Qwen3-1.7B linear shapes at M = 8192 tokens: (tokens, in, out)
+FULL = {
+    "qkv": (8192, 2048, 4096),
+    "o": (8192, 2048, 2048),
+    "gate_up": (8192, 2048, 12288),
+    "down": (8192, 6144, 2048),
+}
+
+
+@pytest.mark.parametrize("name", list(FULL))
+@pytest.mark.parametrize("mode", [FPROP, DGRAD, WGRAD])
+def test_gemm_full_size_sampled(name, mode):
+    T, Din, Dout = FULL[name]
+    X, W, dY = _layer(T, Din, Dout, seed=hash(name) % 1000 + 10 * mode)
+    M = {FPROP: T, DGRAD: T, WGRAD: Dout}[mode]
+    rows = _rows(M, 24)
+    y, y_ref, asum = _run_mode(mode, X, W, dY, rows=rows)
+    check_gemm(y, y_ref, asum, f"{name} mode {mode}")
+
+
+@pytest.mark.parametrize("mode", [FPROP, DGRAD, WGRAD])
+def test_gemm_zero_and_degenerate_inputs(mode):
+    """All-zero activations give an exactly zero output; a single nonzero group
+    gives a rank-one result the oracle reproduces."""
+    T, Din, Dout = 256, 384, 512
+    X, W, dY = _layer(T, Din, Dout, seed=5)
+    Xz = np.zeros_like(X)
+    dYz = np.zeros_like(dY)
+    y, y_ref, asum = _run_mode(mode, Xz, W, dYz)
+    assert np.all(y == 0) and np.all(y_ref == 0)
+    X1 = Xz.copy(); X1[3, 128:256] = X[3, 128:256]
+    dY1 = dYz.copy(); dY1[3, :128] = dY[3, :128]
+    y, y_ref, asum = _run_mode(mode, X1, W, dY1)
+    check_gemm(y, y_ref, asum, f"mode {mode} one group")
+
+
+def test_gemm_deterministic():
+    X, W, dY = _layer(1024, 2048, 2048, seed=9)
+    qx, sx = fp8_quant_act(to_dev_bf16(X))
+    qw, sw, _ = fp8_quant_weight(to_dev_bf16(W))
+    y1 = fp8_gemm_blockwise(FPROP, qx, sx, qw, sw, 1024, 2048, 2048)
+    y2 = fp8_gemm_blockwise(FPROP, qx, sx, qw, sw, 1024, 2048, 2048)
+    assert torch.equal(y1.view(torch.int16), y2.view(torch.int16))
