@@ -1,0 +1,520 @@
+#!/usr/bin/env python
+"""Benchmark of the blockwise-FP8 linear layer (quantize + GEMM) on B200.
+
+One step = one pass of the whole hot path over the four linear layers of a
+Qwen3-1.7B transformer block at M = 8192 tokens (micro-batch 2 x sequence 4096):
+QKV (2048 -> 4096), O (2048 -> 2048), gate/up (2048 -> 12288), down (6144 -> 2048).
+For each linear: fp8_quant_act(X), fp8_quant_weight(W), fprop; fp8_quant_act(dY),
+dgrad; fp8_quant_act_t(dY), fp8_quant_act_t(X), wgrad -- 32 kernel launches, 2.47
+TFLOP of GEMM work.  The metric is TFLOP/s of the whole step (2MNK summed over the
+12 GEMMs, divided by the time of all quantizers and GEMMs).
+
+Inputs are seeded synthetic BF16 tensors (X ~ N(0,1) with 1% outlier channels x20,
+W ~ N(0,0.02), dY ~ N(0,1e-3)); 637 MB per step, larger than the 126 MB L2, so no
+flush is needed between steps.
+
+Usage:  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+Under torchrun (N > 1) each rank runs an independent replica (weak scaling): the path
+shards by tokens with no exchange in the data path.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+METRIC = "blockwise-FP8 linear TFLOP/s (quant+GEMM, M=8192) and % of B200 FP8 peak"
+UNIT = "TFLOP/s"
+TOKENS = 8192
+LINEARS = [("qkv", 2048, 4096), ("o", 2048, 2048), ("gate_up", 2048, 12288), ("down", 6144, 2048)]
+WORKLOAD = "qwen3-1.7b block linears (qkv, o, gate_up, down) fprop+dgrad+wgrad, M=8192"
+STEP_FLOPS = sum(3 * 2 * TOKENS * din * dout for _, din, dout in LINEARS)
+LAUNCHES_PER_STEP = 8 * len(LINEARS)
+FP8_OVER_BF16 = 4.5 / 2.25  # nominal dense FP8 : BF16 tensor throughput on B200
+
+
+def config_dict(n):
+    return {
+        "workload": WORKLOAD,
+        "tokens": TOKENS,
+        "linears": {name: [din, dout] for name, din, dout in LINEARS},
+        "passes": "fprop+dgrad+wgrad with all quantizers",
+        "step_gflop": round(STEP_FLOPS / 1e9, 3),
+        "l2": "inputs larger than L2 (637 MB of BF16 inputs per step), no flush",
+        "parallelism": f"replicas x{n}" if n > 1 else "single GPU",
+    }
+
+
+# --------------------------------------------------------------------- helpers
+
+def dist_env():
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return world, rank, local
+
+
+def measured_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            return json.load(f), "measured"
+    except (OSError, ValueError):
+        return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0}, "fallback"
+
+
+class ClockSampler:
+    """nvidia-smi clock / throttle sampling while the timed region runs."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index):
+        self.gpu = gpu_index
+        self.proc = None
+        self.file = None
+
+    def __enter__(self):
+        self.file = tempfile.NamedTemporaryFile("w+", suffix=".csv", delete=False)
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=self.file, stderr=subprocess.DEVNULL)
+        except OSError:
+            self.proc = None
+        time.sleep(0.3)
+        return self
+
+    def __exit__(self, *exc):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+        self.file.flush()
+
+    def summary(self):
+        rows = []
+        try:
+            with open(self.file.name) as f:
+                for line in f:
+                    parts = [p.strip() for p in line.split(",")]
+                    if len(parts) >= 9:
+                        rows.append(parts)
+        finally:
+            os.unlink(self.file.name)
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unavailable"]}
+        sm = [float(r[1]) for r in rows if r[1].replace(".", "").isdigit()]
+        smax = [float(r[2]) for r in rows if r[2].replace(".", "").isdigit()]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in rows for i in range(4) if r[5 + i] == "Active"})
+        loaded = [v for v in sm if v > 0.5 * (max(smax) if smax else 0)] or sm
+        return {"sm_mhz": statistics.median(loaded) if loaded else None,
+                "sm_max_mhz": max(smax) if smax else None,
+                "reasons": reasons, "samples": len(rows)}
+
+
+# ------------------------------------------------------------------- our arm
+
+class LayerWork:
+    """Device buffers of one step and the launch sequence through the C ABI."""
+
+    def __init__(self, dev, host_inputs):
+        import torch
+        import blockwise_fp8_linear_b200 as fb
+        self.fb = fb
+        self.torch = torch
+        self.lin = []
+        for (name, din, dout), (X, W, dY) in zip(LINEARS, host_inputs):
+            t = lambda a: torch.from_numpy(a.view(np.int16)).view(torch.bfloat16)
+            d = {
+                "name": name, "din": din, "dout": dout,
+                "X": t(X).to(dev), "W": t(W).to(dev), "dY": t(dY).to(dev),
+                "qx": torch.empty(TOKENS, din, dtype=torch.uint8, device=dev),
+                "sx": torch.empty(din // 128, TOKENS, dtype=torch.float32, device=dev),
+                "qw": torch.empty(dout, din, dtype=torch.uint8, device=dev),
+                "sw": torch.empty(dout // 128, din // 128, dtype=torch.float32, device=dev),
+                "qdy": torch.empty(TOKENS, dout, dtype=torch.uint8, device=dev),
+                "sdy": torch.empty(dout // 128, TOKENS, dtype=torch.float32, device=dev),
+                "qdyt": torch.empty(dout, TOKENS, dtype=torch.uint8, device=dev),
+                "sdyt": torch.empty(TOKENS // 128, dout, dtype=torch.float32, device=dev),
+                "qxt": torch.empty(din, TOKENS, dtype=torch.uint8, device=dev),
+                "sxt": torch.empty(TOKENS // 128, din, dtype=torch.float32, device=dev),
+                "Y": torch.empty(TOKENS, dout, dtype=torch.bfloat16, device=dev),
+                "dX": torch.empty(TOKENS, din, dtype=torch.bfloat16, device=dev),
+                "dW": torch.empty(dout, din, dtype=torch.bfloat16, device=dev),
+            }
+            self.lin.append(d)
+        self.h2d_bytes = sum(d[k].numel() * 2 for d in self.lin for k in ("X", "W", "dY"))
+        self.d2h_bytes = sum(d[k].numel() * 2 for d in self.lin for k in ("Y", "dX", "dW"))
+
+    def step(self, gemm_events=None):
+        """Enqueue one step on the current stream.  gemm_events: optional list that
+        receives (start, end, flops) CUDA-event triples around each GEMM."""
+        fb, torch = self.fb, self.torch
+        L = fb.lib()
+        st = fb._stream(None)
+        T = TOKENS
+
+        def gemm(mode, a, sa, b, sb, out, M, N, K):
+            if gemm_events is not None:
+                e0 = torch.cuda.Event(enable_timing=True)
+                e1 = torch.cuda.Event(enable_timing=True)
+                e0.record()
+            rc = L.fp8_gemm_blockwise(mode, a.data_ptr(), sa.data_ptr(), b.data_ptr(),
+                                      sb.data_ptr(), out.data_ptr(), M, N, K, st)
+            if rc:
+                raise fb.Fp8bwError(rc, "fp8_gemm_blockwise")
+            if gemm_events is not None:
+                e1.record()
+                gemm_events.append((e0, e1, 2 * M * N * K))
+
+        def chk(rc, what):
+            if rc:
+                raise fb.Fp8bwError(rc, what)
+
+        for d in self.lin:
+            din, dout = d["din"], d["dout"]
+            chk(L.fp8_quant_act(d["X"].data_ptr(), T, din, d["qx"].data_ptr(), d["sx"].data_ptr(), st), "qa")
+            chk(L.fp8_quant_weight(d["W"].data_ptr(), dout, din, d["qw"].data_ptr(),
+                                   d["sw"].data_ptr(), None, st), "qw")
+            gemm(fb.FPROP, d["qx"], d["sx"], d["qw"], d["sw"], d["Y"], T, dout, din)
+            chk(L.fp8_quant_act(d["dY"].data_ptr(), T, dout, d["qdy"].data_ptr(), d["sdy"].data_ptr(), st), "qa")
+            gemm(fb.DGRAD, d["qdy"], d["sdy"], d["qw"], d["sw"], d["dX"], T, din, dout)
+            chk(L.fp8_quant_act_t(d["dY"].data_ptr(), T, dout, d["qdyt"].data_ptr(), d["sdyt"].data_ptr(), st), "qt")
+            chk(L.fp8_quant_act_t(d["X"].data_ptr(), T, din, d["qxt"].data_ptr(), d["sxt"].data_ptr(), st), "qt")
+            gemm(fb.WGRAD, d["qdyt"], d["sdyt"], d["qxt"], d["sxt"], d["dW"], dout, din, T)
+
+
+def make_inputs(rank=0):
+    from blockwise_fp8_linear_b200 import synth
+    out = []
+    for i, (name, din, dout) in enumerate(LINEARS):
+        wl = 10 + i
+        X = synth.normal_bf16(TOKENS, din, 1.0, seed=synth.seed_for(wl, 0 + 10 * rank), outliers=True)
+        W = synth.normal_bf16(dout, din, 0.02, seed=synth.seed_for(wl, 1))
+        dY = synth.normal_bf16(TOKENS, dout, 1e-3, seed=synth.seed_for(wl, 2 + 10 * rank))
+        out.append((X, W, dY))
+    return out
+
+
+def barrier(world):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+def max_over_ranks(x, world):
+    if world == 1:
+        return x
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def run_ours(args):
+    import torch
+    world, rank, local = dist_env()
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+    dev = torch.device("cuda", local if world > 1 else 0)
+    torch.cuda.set_device(dev)
+    from blockwise_fp8_linear_b200 import build as fbuild
+    fbuild.build()
+    import blockwise_fp8_linear_b200 as fb
+
+    host = make_inputs(rank)
+    work = LayerWork(dev, host)
+
+    # warm-up
+    for _ in range(args.warmup):
+        work.step()
+    torch.cuda.synchronize()
+    if fb.fp8bw_last_device_error() != 0:
+        raise RuntimeError("a bounded in-kernel wait ran out during warm-up")
+
+    # timed region: K steps, device time by CUDA events, GEMM launches bracketed
+    gemm_events = []
+    with ClockSampler(dev.index) as clocks:
+        barrier(world)
+        torch.cuda.synchronize()
+        t0 = torch.cuda.Event(enable_timing=True)
+        t1 = torch.cuda.Event(enable_timing=True)
+        t0.record()
+        for _ in range(args.steps):
+            work.step(gemm_events)
+        t1.record()
+        torch.cuda.synchronize()
+        barrier(world)
+    local_ms = t0.elapsed_time(t1)
+    elapsed_ms = max_over_ranks(local_ms, world)
+    if fb.fp8bw_last_device_error() != 0:
+        raise RuntimeError("a bounded in-kernel wait ran out in the timed region")
+    gemm_ms = sum(e0.elapsed_time(e1) for e0, e1, _ in gemm_events)
+    gemm_flops = sum(f for _, _, f in gemm_events)
+    clock_info = clocks.summary()
+
+    ms_per_step = elapsed_ms / args.steps
+    value = world * STEP_FLOPS / (ms_per_step * 1e-3) / 1e12
+
+    # end to end through the public API: pinned host inputs -> device, step,
+    # results -> pinned host, all inside the timed region
+    e2e = None
+    if not args.no_e2e:
+        pin_in = [(torch.from_numpy(X.view(np.int16)).pin_memory(),
+                   torch.from_numpy(W.view(np.int16)).pin_memory(),
+                   torch.from_numpy(dY.view(np.int16)).pin_memory()) for X, W, dY in host]
+        pin_out = [(torch.empty(d["Y"].shape, dtype=torch.int16).pin_memory(),
+                    torch.empty(d["dX"].shape, dtype=torch.int16).pin_memory(),
+                    torch.empty(d["dW"].shape, dtype=torch.int16).pin_memory()) for d in work.lin]
+
+        def e2e_step():
+            for d, (X, W, dY) in zip(work.lin, pin_in):
+                d["X"].view(torch.int16).copy_(X, non_blocking=True)
+                d["W"].view(torch.int16).copy_(W, non_blocking=True)
+                d["dY"].view(torch.int16).copy_(dY, non_blocking=True)
+            work.step()
+            for d, (Y, dX, dW) in zip(work.lin, pin_out):
+                Y.copy_(d["Y"].view(torch.int16), non_blocking=True)
+                dX.copy_(d["dX"].view(torch.int16), non_blocking=True)
+                dW.copy_(d["dW"].view(torch.int16), non_blocking=True)
+
+        e2e_step()
+        torch.cuda.synchronize()
+        n_e2e = max(3, min(args.steps, 20))
+        barrier(world)
+        a0 = torch.cuda.Event(enable_timing=True)
+        a1 = torch.cuda.Event(enable_timing=True)
+        a0.record()
+        for _ in range(n_e2e):
+            e2e_step()
+        a1.record()
+        torch.cuda.synchronize()
+        barrier(world)
+        e2e_ms = max_over_ranks(a0.elapsed_time(a1), world) / n_e2e
+        e2e = {"value": round(world * STEP_FLOPS / (e2e_ms * 1e-3) / 1e12, 3), "unit": UNIT,
+               "h2d_bytes_per_step": work.h2d_bytes, "d2h_bytes_per_step": work.d2h_bytes,
+               "ms_per_step": round(e2e_ms, 4), "steps": n_e2e}
+
+    peaks, peak_src = measured_peaks()
+    fp8_peak = peaks["bf16_tflops"] * FP8_OVER_BF16
+    achieved = gemm_flops / (gemm_ms * 1e-3) / 1e12
+    roofline = {
+        "kernel": "fp8_gemm_kernel (fprop/dgrad/wgrad, all 12 GEMMs of the step)",
+        "bound": "tensor", "achieved": round(achieved, 2),
+        "peak": round(fp8_peak, 1), "unit": "TFLOP/s", "frac": round(achieved / fp8_peak, 4),
+        "peak_source": f"{peak_src} cuBLAS bf16 burst x {FP8_OVER_BF16:g} (nominal FP8:BF16)",
+        "traffic": None,
+        "gemm_share_of_step": round(gemm_ms / local_ms, 4),
+    }
+
+    cpu = None
+    if rank == 0 and not args.no_cpu:
+        cpu = cpu_baseline(budget_s=args.cpu_budget, host=host)
+
+    if rank == 0:
+        line = {
+            "metric": METRIC, "value": round(value, 3), "unit": UNIT, "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_per_step, 4),
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "dtype": "e4m3", "data": "synthetic (seeded splitmix64/Box-Muller BF16)",
+            "config": config_dict(world), "roofline": roofline, "cpu_baseline": cpu,
+            "e2e": e2e, "gpu_launches": LAUNCHES_PER_STEP * args.steps,
+            "clocks": clock_info,
+            "pct_of_fp8_peak": round(100 * value / world / fp8_peak, 2),
+        }
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+
+
+# ----------------------------------------------------- oracle (CPU) timing
+
+def oracle_sample_step(i, host, threads):
+    """One bounded sample of the step on the CPU oracle: linear i % 4, GEMM mode
+    (i // 4) % 3, one 128-row tile of the output, with the quantization of exactly
+    the groups that tile reads.  Returns (GEMM flops done, seconds)."""
+    import oracle
+    li = i % len(LINEARS)
+    mode = (i // len(LINEARS)) % 3
+    name, din, dout = LINEARS[li]
+    X, W, dY = host[li]
+    r0 = 128 * ((i // 12) % (TOKENS // 128))
+    t = time.perf_counter()
+    if mode == oracle.FPROP:
+        a, sa = oracle.quant_act(np.ascontiguousarray(X[r0:r0 + 128]))
+        b, sb, _ = oracle.quant_weight(W)
+        M, N, K = 128, dout, din
+    elif mode == oracle.DGRAD:
+        a, sa = oracle.quant_act(np.ascontiguousarray(dY[r0:r0 + 128]))
+        b, sb, _ = oracle.quant_weight(W)
+        M, N, K = 128, din, dout
+    else:
+        # output rows r0..r0+127 of dW (out-features): those columns of dY, all tokens
+        a, sa = oracle.quant_act_t(np.ascontiguousarray(dY[:, r0 % dout:(r0 % dout) + 128]))
+        b, sb = oracle.quant_act_t(X)
+        M, N, K = 128, din, TOKENS
+    oracle.gemm(mode, a, sa, b, sb, M, N, K, nthreads=threads)
+    return 2 * M * N * K, time.perf_counter() - t
+
+
+def cpu_baseline(budget_s=15.0, host=None, max_steps=None):
+    import oracle
+    threads = oracle.max_threads()
+    if host is None:
+        host = make_inputs(0)
+    flops = 0
+    secs = 0.0
+    n = 0
+    while secs < budget_s and (max_steps is None or n < max_steps):
+        f, s = oracle_sample_step(n, host, threads)
+        flops += f
+        secs += s
+        n += 1
+    return {"value": round(flops / secs / 1e12, 6), "unit": UNIT, "cores": threads,
+            "kind": "oracle",
+            "sample": f"{n} samples, each one 128-row output tile of one of the 12 GEMMs of the "
+                      f"step (rotating linear x mode) plus the oracle quantization of the groups "
+                      f"it reads; FP64 GEMM, {threads} OpenMP threads, {secs:.1f} s"}
+
+
+def run_reference(args):
+    world, rank, _ = dist_env()
+    if rank != 0:
+        return
+    import oracle
+    threads = oracle.max_threads()
+    host = make_inputs(0)
+    for i in range(args.warmup):
+        oracle_sample_step(i, host, threads)
+    flops = 0
+    secs = 0.0
+    for i in range(args.steps):
+        f, s = oracle_sample_step(args.warmup + i, host, threads)
+        flops += f
+        secs += s
+    value = flops / secs / 1e12
+    line = {
+        "impl": "reference", "metric": METRIC, "value": round(value, 6), "unit": UNIT,
+        "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": round(1e3 * secs / args.steps, 3), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": config_dict(world),
+        "cpu_baseline": {"value": round(value, 6), "unit": UNIT, "cores": threads, "kind": "oracle",
+                         "sample": "each step: one 128-row output tile of one of the 12 GEMMs "
+                                   "(rotating), with the quantization of the groups it reads"},
+        "e2e": {"value": round(value, 6), "unit": UNIT, "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+KERNEL_CASES = ("gemm_fprop", "gemm_dgrad", "gemm_wgrad", "quant_act", "quant_act_t",
+                "quant_weight")
+
+
+def run_kernel_only(args):
+    """Launch one kernel of the step (QKV linear shapes: M=8192, 2048 -> 4096; the
+    quantizers on the 8192x12288 gate/up gradient so inputs exceed L2) warmup+steps
+    times back to back and print its mean device time.  For profilers."""
+    import torch
+    import blockwise_fp8_linear_b200 as fb
+    from blockwise_fp8_linear_b200 import build as fbuild
+    fbuild.build()
+    dev = torch.device("cuda", 0)
+    g = torch.Generator(device=dev).manual_seed(0)
+    T, din, dout = TOKENS, 2048, 4096
+    case = args.kernel_only
+
+    def randn(r, c, std):
+        return (torch.randn(r, c, device=dev, generator=g) * std).to(torch.bfloat16)
+
+    if case.startswith("gemm"):
+        X, W, dY = randn(T, din, 1.0), randn(dout, din, 0.02), randn(T, dout, 1e-3)
+        qw, sw, _ = fb.fp8_quant_weight(W)
+        if case == "gemm_fprop":
+            a, sa = fb.fp8_quant_act(X)
+            launch = lambda: fb.fp8_gemm_blockwise(fb.FPROP, a, sa, qw, sw, T, dout, din)
+            flops = 2 * T * din * dout
+        elif case == "gemm_dgrad":
+            a, sa = fb.fp8_quant_act(dY)
+            launch = lambda: fb.fp8_gemm_blockwise(fb.DGRAD, a, sa, qw, sw, T, din, dout)
+            flops = 2 * T * din * dout
+        else:
+            a, sa = fb.fp8_quant_act_t(dY)
+            b, sb = fb.fp8_quant_act_t(X)
+            launch = lambda: fb.fp8_gemm_blockwise(fb.WGRAD, a, sa, b, sb, dout, din, T)
+            flops = 2 * T * din * dout
+        work = ("TFLOP/s", flops / 1e12)
+    else:
+        R, C = T, 12288
+        X = randn(R, C, 1.0)
+        if case == "quant_act":
+            launch = lambda: fb.fp8_quant_act(X)
+        elif case == "quant_act_t":
+            launch = lambda: fb.fp8_quant_act_t(X)
+        else:
+            launch = lambda: fb.fp8_quant_weight(X)
+        work = ("GB/s", R * C * (3 + 4 / 128) / 1e9)
+    torch.cuda.synchronize()
+    for _ in range(args.warmup):
+        launch()
+    torch.cuda.synchronize()
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(args.steps):
+        launch()
+    e1.record()
+    torch.cuda.synchronize()
+    ms = e0.elapsed_time(e1) / args.steps
+    print(json.dumps({"kernel_only": case, "ms": round(ms, 5),
+                      work[0]: round(work[1] / (ms * 1e-3), 2)}), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser(description=__doc__.split("\n\n")[0])
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu", action="store_true")
+    ap.add_argument("--cpu-budget", type=float, default=15.0, help="seconds of oracle work")
+    ap.add_argument("--kernel-only", choices=KERNEL_CASES, default=None,
+                    help="launch one kernel repeatedly (for profilers); no JSON metric line")
+    args = ap.parse_args()
+    if args.kernel_only:
+        run_kernel_only(args)
+        return
+    if args.warmup < 3 and args.impl == "ours":
+        ap.error("--warmup must be >= 3")
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_ours(args)
+
+
+if __name__ == "__main__":
+    main()

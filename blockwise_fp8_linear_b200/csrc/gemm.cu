@@ -6,23 +6,35 @@
 // section 3.2: all three GEMMs use the FP8 path, with FP32 accumulation and a BF16
 // result handed back to the model).
 //
-// Design (one persistent CTA per SM, warp-specialised):
-//   warp 0      TMA producer: 128x128 A tile + BNx128 B tile per stage, 128-byte
-//               swizzle, STAGES-deep ring of shared-memory stages.
-//   warp 1      MMA issuer: per reduction block, 4 x tcgen05.mma kind::f8f6f4
-//               (K = 32 each) into one of two TMEM partial buffers (fresh
-//               accumulation per block), then commits to the stage's "empty" barrier
-//               and to the buffer's "full" barrier.
-//   warps 2..3  idle (they complete the first warpgroup, which gives registers away)
+// Design (persistent, warp-specialised, one CTA per SM):
+//   warp 0      TMA producer: per reduction block one 128x128 A tile and one B tile
+//               (128B swizzle) into a STAGES-deep ring of shared-memory stages.
+//   warp 1      MMA issuer: per reduction block 4 x tcgen05.mma kind::f8f6f4 (K = 32
+//               bytes each) into one of two TMEM partial buffers (fresh accumulation
+//               per block), then commits to the stage's "empty" barrier and to the
+//               buffer's "full" barrier.
+//   warp 2      scale loader: copies each reduction block's scales (a-scales of the
+//               CTA's rows, b-scales of the tile) into a shared-memory ring with
+//               cp.async, signalling a per-slot barrier when they land.
+//   warp 3      idle (completes the first warpgroup, which gives registers away)
 //   warps 4..11 promotion + epilogue: each thread owns one TMEM lane (a row of the
-//               tile) and COLS columns.  Per block it loads the FP32 partial from TMEM,
-//               releases the buffer, and adds partial * scale into an FP32 running sum
-//               held in registers (packed f32x2 FMA).  After the last block it rounds
-//               the sum to BF16 and stores it.
+//               tile) and COLS columns.  Per block it loads the FP32 partial from
+//               TMEM 32 columns at a time, releases the buffer, and adds partial x
+//               scale into an FP32 running sum held in registers (packed f32x2
+//               FMA).  After the last block it rounds the sum to BF16 and stores it.
 // Double-buffered TMEM partials let the tensor cores run block kb+1 while the
-// epilogue promotes block kb.  Every wait is bounded (about one second); a wait that
-// runs out records an error code and the whole block unwinds.
+// epilogue promotes block kb.
+//
+// CTA pairs (CG = 2, when M is a multiple of 256): a cluster of two CTAs computes a
+// 256 x BN tile with tcgen05.mma.cta_group::2 issued by the even CTA.  Each CTA
+// loads its own 128 rows of A and its own BN/2 columns of B (no multicast), and holds
+// its 128 rows of D in its own TMEM, so per SM the shared-memory and L2 operand
+// traffic per FLOP drops by a third against one CTA computing 128 x BN.
+//
+// Every wait is bounded (about one second); a wait that runs out records an error
+// code in a device word and the whole CTA (pair) unwinds.
 #include <cstdint>
+#include <cstring>
 #include <cuda.h>
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
@@ -34,18 +46,20 @@ namespace fp8bw {
 
 __device__ int g_device_error;  // first error code seen by a bounded wait (0 = none)
 
-constexpr int BM = 128;
-constexpr int BK = 128;
+constexpr int BM = 128;  // rows of D per CTA
+constexpr int BK = 128;  // one reduction block
 constexpr uint64_t WAIT_LIMIT_NS = 1000000000ull;
-constexpr uint64_t DRAIN_LIMIT_NS = 100000000ull;
+constexpr uint64_t DRAIN_NS = 20000000ull;
 
-enum : int { ERR_PRODUCER = 1, ERR_MMA_FULL = 2, ERR_MMA_TEMPTY = 3, ERR_EPI = 4, ERR_DRAIN = 5 };
+enum : int { ERR_PRODUCER = 1, ERR_MMA_FULL = 2, ERR_MMA_TEMPTY = 3, ERR_EPI = 4, ERR_SCALES = 5 };
 
-template <int BN_, int MODE_, int STAGES_>
+template <int BN_, int MODE_, int STAGES_, int CG_>
 struct GemmCfg {
-    static constexpr int BN = BN_;
+    static constexpr int BN = BN_;      // columns of D per tile (both CTAs of a pair)
     static constexpr int MODE = MODE_;  // 0 fprop, 1 dgrad (B is MN-major), 2 wgrad
     static constexpr int STAGES = STAGES_;
+    static constexpr int CG = CG_;      // CTAs per MMA (1 or 2)
+    static constexpr int TILE_M = BM * CG;
     static constexpr int EPI_WARPS = 8;
     static constexpr int COLS = 4 * BN / EPI_WARPS;  // columns per epilogue thread
     static constexpr int THREADS = 128 + 32 * EPI_WARPS;  // 3 warpgroups
@@ -56,15 +70,38 @@ struct GemmCfg {
     static constexpr int REGS_LOW = 72;
     static constexpr int REGS_HIGH = 216;
     static constexpr int REGS_NEEDED = 128 * REGS_LOW + 32 * EPI_WARPS * REGS_HIGH;
+    static constexpr int B_ROWS = BN / CG;  // B rows (N) this CTA loads per stage
     static constexpr int A_BYTES = BM * BK;
-    static constexpr int B_BYTES = BN * BK;
+    static constexpr int B_BYTES = B_ROWS * BK;
     static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
-    static constexpr int TMEM_COLS = 2 * BN;
-    static constexpr int SBV_BYTES = (MODE == 2) ? EPI_WARPS * COLS * 4 : 0;
-    static constexpr int BAR_OFF = STAGES * STAGE_BYTES + SBV_BYTES;
-    static constexpr int SMEM = 1024 + BAR_OFF + 256;
+    // TMEM holds NBUF partial buffers of BN fp32 columns (512 columns in all), so the
+    // MMA can run NBUF-1 reduction blocks ahead of the promotion.
+    static constexpr int NBUF = 512 / BN;
+    static constexpr int TMEM_COLS = 512;
+    // MN-major B (dgrad) boxes: 128 N-bytes with the 128-byte swizzle, or 64 with the
+    // 64-byte swizzle when this CTA holds only 64 columns of B.
+    static constexpr int B_BOX = (B_ROWS >= 128) ? 128 : 64;
+    // Scale ring shared by the CTA, filled by the scale-loader warp: one slot per
+    // (tile, reduction block) with the a-scales of the CTA's 128 rows and the
+    // b-scale(s) of the tile: BN/128 block scales (fprop/dgrad) or BN column scales
+    // (wgrad).
+    static constexpr int SRING = 8;
+    static constexpr int SB_FLOATS = (MODE == 2) ? BN : 4;
+    static constexpr int SLOT_FLOATS = BM + SB_FLOATS;
+    static constexpr int RING_BYTES = SRING * SLOT_FLOATS * 4;
+    static_assert((SLOT_FLOATS * 4) % 16 == 0, "scale slots must stay 16-byte aligned");
+    // Pair path: the finished tile leaves through shared memory and TMA bulk
+    // stores; each epilogue warp owns 32 rows x COLS columns of BF16 staging, laid
+    // out as 64-column boxes of 32 rows x 128 B with the 128-byte swizzle.
+    static constexpr bool TMA_STORE = (CG == 2);
+    static constexpr int STAGE_OUT_WARP = 32 * COLS * 2;
+    static constexpr int OUT_BYTES = TMA_STORE ? EPI_WARPS * STAGE_OUT_WARP : 0;
+    static constexpr int RING_OFF = STAGES * STAGE_BYTES + OUT_BYTES;
+    static constexpr int BAR_OFF = RING_OFF + RING_BYTES;
+    static constexpr int SMEM = 1024 + BAR_OFF + 512;
     static_assert(COLS % 32 == 0, "columns per thread must be whole TMEM load chunks");
     static_assert(BN % 128 == 0 && BN <= 256, "BN must be 128 or 256");
+    static_assert(B_ROWS % B_BOX == 0, "B rows must be whole boxes");
     static_assert(SMEM <= 227 * 1024, "shared memory budget");
 };
 
@@ -86,26 +123,32 @@ __device__ __forceinline__ void tile_coords(int t, int tiles_m, int tiles_n, int
 template <class Cfg>
 __global__ void __launch_bounds__(Cfg::THREADS, 1)
 fp8_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
-                const float *__restrict__ sa, const float *__restrict__ sb,
+                const __grid_constant__ CUtensorMap tmD, const float *__restrict__ sa, const float *__restrict__ sb,
                 __nv_bfloat16 *__restrict__ D, int M, int N, int K)
 {
-    constexpr int BN = Cfg::BN, MODE = Cfg::MODE, STAGES = Cfg::STAGES;
+    constexpr int BN = Cfg::BN, MODE = Cfg::MODE, STAGES = Cfg::STAGES, CG = Cfg::CG;
     constexpr int COLS = Cfg::COLS, EPI_WARPS = Cfg::EPI_WARPS;
 
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-    float *sbv = reinterpret_cast<float *>(smem + STAGES * Cfg::STAGE_BYTES);
+    uint8_t *sout = smem + STAGES * Cfg::STAGE_BYTES;
+    float *sring = reinterpret_cast<float *>(smem + Cfg::RING_OFF);
     uint64_t *bars = reinterpret_cast<uint64_t *>(smem + Cfg::BAR_OFF);
-    uint64_t *full = bars;                 // [STAGES] TMA -> MMA
+    uint64_t *full = bars;                 // [STAGES] TMA -> MMA   (used in the even CTA)
     uint64_t *empty = bars + STAGES;       // [STAGES] MMA -> TMA
-    uint64_t *tfull = bars + 2 * STAGES;   // [2] MMA -> epilogue
-    uint64_t *tempty = tfull + 2;          // [2] epilogue -> MMA
-    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(tempty + 2);
+    uint64_t *tfull = bars + 2 * STAGES;   // [NBUF] MMA -> epilogue
+    uint64_t *tempty = tfull + Cfg::NBUF;  // [NBUF] epilogue -> MMA   (used in the even CTA)
+    uint64_t *sfull = tempty + Cfg::NBUF;  // [SRING] scale loader -> epilogue
+    uint64_t *sempty = sfull + Cfg::SRING; // [SRING] epilogue -> scale loader
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(sempty + Cfg::SRING);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int tiles_m = M / BM, tiles_n = N / BN;
+    const int rank = (CG == 2) ? int(cluster_ctarank()) : 0;
+    const int unit = (CG == 2) ? int(cluster_id_x()) : int(blockIdx.x);      // tile walker
+    const int units = (CG == 2) ? int(cluster_count_x()) : int(gridDim.x);
+    const int tiles_m = M / Cfg::TILE_M, tiles_n = N / BN;
     const int num_tiles = tiles_m * tiles_n;
     const int KB = K / BK;
 
@@ -114,9 +157,13 @@ fp8_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__
             mbar_init(&full[s], 1);
             mbar_init(&empty[s], 1);
         }
-        for (int b = 0; b < 2; ++b) {
+        for (int b = 0; b < Cfg::NBUF; ++b) {
             mbar_init(&tfull[b], 1);
-            mbar_init(&tempty[b], EPI_WARPS);
+            mbar_init(&tempty[b], EPI_WARPS * CG);
+        }
+        for (int r = 0; r < Cfg::SRING; ++r) {
+            mbar_init(&sfull[r], 32);
+            mbar_init(&sempty[r], EPI_WARPS);
         }
         *abort_flag = 0;
         fence_mbarrier_init();
@@ -124,46 +171,63 @@ fp8_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__
         tma_prefetch_desc(&tmB);
     }
     if (warp == 1) {
-        tmem_alloc(tmem_slot, Cfg::TMEM_COLS);
-        tmem_relinquish();
+        tmem_alloc<CG>(tmem_slot, Cfg::TMEM_COLS);
+        tmem_relinquish<CG>();
     }
     tc_fence_before();
-    __syncthreads();
+    if (CG == 2)
+        cluster_sync();  // barriers of both CTAs initialised before any remote arrive
+    else
+        __syncthreads();
     tc_fence_after();
     const uint32_t tmem_base = *tmem_slot;
-
-    // Producer / MMA state kept for the drain after an abort.
-    uint32_t armed_mask = 0, armed_parity = 0;  // producer: stages with a load in flight
-    int last_buf = -1;
-    uint32_t last_tparity = 0;                  // MMA: last commit to tfull
+    // cluster-window addresses of the even CTA's barriers
+    const uint32_t full_lead = (CG == 2) ? mapa_shared(smem_u32(full), 0) : smem_u32(full);
+    const uint32_t tempty_lead = (CG == 2) ? mapa_shared(smem_u32(tempty), 0) : smem_u32(tempty);
 
     if (warp < Cfg::EPI_WARP0) {
-      regs_dec<Cfg::REGS_LOW>();
-      if (warp == 0) {
-        if (lane == 0) {
+        regs_dec<Cfg::REGS_LOW>();
+        if (warp == 0 && lane == 0) {
+            // ---------------------------------------------------------- producer
             int stage = 0;
             uint32_t phase = 0;
-            for (int t = blockIdx.x; t < num_tiles && !*abort_flag; t += gridDim.x) {
+            for (int t = unit; t < num_tiles && !*abort_flag; t += units) {
                 int tm, tn;
                 tile_coords(t, tiles_m, tiles_n, tm, tn);
+                const int arow = tm * Cfg::TILE_M + rank * BM;
+                const int bcol = tn * BN + rank * Cfg::B_ROWS;
                 for (int kb = 0; kb < KB; ++kb) {
                     if (!mbar_wait_bounded(&empty[stage], phase ^ 1u, abort_flag, &g_device_error,
                                            ERR_PRODUCER, WAIT_LIMIT_NS))
-                        goto producer_done;
+                        goto role_done;
                     uint8_t *sA = smem + stage * Cfg::STAGE_BYTES;
                     uint8_t *sB = sA + Cfg::A_BYTES;
-                    mbar_arrive_expect_tx(&full[stage], Cfg::STAGE_BYTES);
-                    armed_mask |= 1u << stage;
-                    armed_parity = (armed_parity & ~(1u << stage)) | (phase << stage);
-                    tma_load_2d(sA, &tmA, &full[stage], kb * BK, tm * BM);
-                    if (MODE == 1) {
-                        // B = W[K][N] with N contiguous: BN/128 boxes of 128 (N) x 128 (K).
+                    if (CG == 1) {
+                        mbar_arrive_expect_tx(&full[stage], Cfg::STAGE_BYTES);
+                        tma_load_2d(sA, &tmA, &full[stage], kb * BK, arow);
+                        if (MODE == 1) {
+                            // B = W[K][N] with N contiguous: boxes of B_BOX (N) x 128 (K).
 #pragma unroll
-                        for (int j = 0; j < BN / 128; ++j)
-                            tma_load_2d(sB + j * 128 * BK, &tmB, &full[stage], tn * BN + j * 128,
-                                        kb * BK);
+                            for (int j = 0; j < Cfg::B_ROWS / Cfg::B_BOX; ++j)
+                                tma_load_2d(sB + j * Cfg::B_BOX * BK, &tmB, &full[stage],
+                                            bcol + j * Cfg::B_BOX, kb * BK);
+                        } else {
+                            tma_load_2d(sB, &tmB, &full[stage], kb * BK, bcol);
+                        }
                     } else {
-                        tma_load_2d(sB, &tmB, &full[stage], kb * BK, tn * BN);
+                        // The even CTA's barrier counts the bytes of both CTAs.
+                        if (rank == 0)
+                            mbar_arrive_expect_tx(&full[stage], 2 * Cfg::STAGE_BYTES);
+                        const uint32_t fb = full_lead + uint32_t(stage) * 8u;
+                        tma_load_2d_pair(sA, &tmA, fb, kb * BK, arow);
+                        if (MODE == 1) {
+#pragma unroll
+                            for (int j = 0; j < Cfg::B_ROWS / Cfg::B_BOX; ++j)
+                                tma_load_2d_pair(sB + j * Cfg::B_BOX * BK, &tmB, fb,
+                                                 bcol + j * Cfg::B_BOX, kb * BK);
+                        } else {
+                            tma_load_2d_pair(sB, &tmB, fb, kb * BK, bcol);
+                        }
                     }
                     if (++stage == STAGES) {
                         stage = 0;
@@ -171,21 +235,19 @@ fp8_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__
                     }
                 }
             }
-        producer_done:;
-        }
-    } else if (warp == 1) {
-        if (lane == 0) {
-            constexpr uint32_t idesc = make_idesc_e4m3(BM, BN, MODE == 1 ? 1 : 0);
+        } else if (warp == 1 && lane == 0 && rank == 0) {
+            // --------------------------------------------------------------- MMA
+            constexpr uint32_t idesc = make_idesc_e4m3(Cfg::TILE_M, BN, MODE == 1 ? 1 : 0);
             int stage = 0, buf = 0;
             uint32_t phase = 0, tphase = 0;
-            for (int t = blockIdx.x; t < num_tiles && !*abort_flag; t += gridDim.x) {
+            for (int t = unit; t < num_tiles && !*abort_flag; t += units) {
                 for (int kb = 0; kb < KB; ++kb) {
                     if (!mbar_wait_bounded(&full[stage], phase, abort_flag, &g_device_error,
                                            ERR_MMA_FULL, WAIT_LIMIT_NS))
-                        goto mma_done;
+                        goto role_done;
                     if (!mbar_wait_bounded(&tempty[buf], tphase ^ 1u, abort_flag, &g_device_error,
                                            ERR_MMA_TEMPTY, WAIT_LIMIT_NS))
-                        goto mma_done;
+                        goto role_done;
                     tc_fence_after();
                     const uint32_t a_addr = smem_u32(smem + stage * Cfg::STAGE_BYTES);
                     const uint32_t b_addr = a_addr + Cfg::A_BYTES;
@@ -196,198 +258,243 @@ fp8_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__
                         // a K step of 32 bytes moves the start address by 32 B.
                         const uint64_t adesc = make_smem_desc_sw128(a_addr + k * 32, 16, 1024);
                         uint64_t bdesc;
-                        if (MODE == 1) {
+                        if (MODE == 1 && Cfg::B_BOX == 128) {
                             // MN-major, 128B swizzle: 128 N-bytes per row, one row per k;
                             // atoms of 8 k-rows 1024 B apart (SBO), 128-wide N atoms
                             // 16 KB apart (LBO); a K step of 32 rows moves 4 KB.
                             bdesc = make_smem_desc_sw128(b_addr + k * 32 * 128, 128 * BK, 1024);
+                        } else if (MODE == 1) {
+                            // MN-major, 64B swizzle: 64 N-bytes per row; atoms of 8 k-rows
+                            // 512 B apart (SBO); a K step of 32 rows moves 2 KB.
+                            bdesc = make_smem_desc_sw64(b_addr + k * 32 * 64, 64 * BK, 512);
                         } else {
                             bdesc = make_smem_desc_sw128(b_addr + k * 32, 16, 1024);
                         }
-                        mma_f8f6f4(d_tmem, adesc, bdesc, idesc, k > 0 ? 1u : 0u);
+                        mma_f8f6f4<CG>(d_tmem, adesc, bdesc, idesc, k > 0 ? 1u : 0u);
                     }
-                    mma_commit(&empty[stage]);
-                    mma_commit(&tfull[buf]);
-                    last_buf = buf;
-                    last_tparity = tphase;
+                    if (CG == 1) {
+                        mma_commit(&empty[stage]);
+                        mma_commit(&tfull[buf]);
+                    } else {
+                        mma_commit_pair(&empty[stage], 0x3);
+                        mma_commit_pair(&tfull[buf], 0x3);
+                    }
                     if (++stage == STAGES) {
                         stage = 0;
                         phase ^= 1u;
                     }
-                    if (++buf == 2) {
+                    if (++buf == Cfg::NBUF) {
                         buf = 0;
                         tphase ^= 1u;
                     }
                 }
             }
-        mma_done:;
+        } else if (warp == 2) {
+            // ------------------------------------------------------ scale loader
+            // All 32 lanes copy one iteration's scales with cp.async; each lane's
+            // copies arrive on the slot's "full" barrier when they land, so the warp
+            // never waits for global memory and runs up to SRING iterations ahead.
+            int j = 0;
+            for (int t = unit; t < num_tiles && !*abort_flag; t += units) {
+                int tm, tn;
+                tile_coords(t, tiles_m, tiles_n, tm, tn);
+                const float *sa_tile = sa + tm * Cfg::TILE_M + rank * BM;
+                const int nb0 = (tn * BN) / 128;
+                for (int kb = 0; kb < KB; ++kb, ++j) {
+                    const int r = j % Cfg::SRING;
+                    const uint32_t ph = uint32_t(j / Cfg::SRING) & 1u;
+                    const bool ok = mbar_wait_bounded(&sempty[r], ph ^ 1u, abort_flag,
+                                                      &g_device_error, ERR_SCALES, WAIT_LIMIT_NS);
+                    if (!__all_sync(0xffffffffu, ok))
+                        goto role_done;
+                    float *slot = sring + r * Cfg::SLOT_FLOATS;
+                    cp_async_16(slot + 4 * lane, sa_tile + size_t(kb) * M + 4 * lane);
+                    if (MODE == 0) {
+                        if (lane < BN / 128)
+                            cp_async_4(slot + BM + lane, sb + size_t(nb0 + lane) * KB + kb);
+                    } else if (MODE == 1) {
+                        if (lane < BN / 128)
+                            cp_async_4(slot + BM + lane, sb + size_t(kb) * (N / 128) + nb0 + lane);
+                    } else {
+                        const float *src = sb + size_t(kb) * N + tn * BN + lane * (BN / 32);
+#pragma unroll
+                        for (int q = 0; q < BN / 128; ++q)
+                            cp_async_16(slot + BM + lane * (BN / 32) + 4 * q, src + 4 * q);
+                    }
+                    cp_async_mbar_arrive(&sfull[r]);
+                }
+            }
+            cp_async_wait<0>();
         }
-      }
+    role_done:;
     } else {
         regs_inc<Cfg::REGS_HIGH>();
         // ---------------------------------------------------- promotion + epilogue
         const int ew = warp - Cfg::EPI_WARP0;
         const int quarter = warp & 3;           // TMEM lanes this warp may access
         const int col0 = (ew >> 2) * COLS;      // columns of the tile this thread owns
-        const int row_in_tile = quarter * 32 + lane;
-        float *my_sbv = sbv + ew * COLS;        // wgrad: this warp's column scales
+        const int row_in_tile = rank * BM + quarter * 32 + lane;
+
+        const int row_local = quarter * 32 + lane;  // the thread's row among the CTA's 128
 
         float2 acc[COLS / 2];
 #pragma unroll
         for (int i = 0; i < COLS / 2; ++i)
             acc[i] = make_float2(0.f, 0.f);
 
-        // Scales of iteration j = (tile index i, block kb), fetched two iterations
-        // ahead.  For fprop/dgrad the thread needs one a-scale (its row) and one
-        // b-scale (its 128-column block); for wgrad one a-scale and COLS b-scales,
-        // which lanes load cooperatively (COLS/32 per lane) into shared memory.
-        constexpr int VB = (MODE == 2) ? COLS / 32 : 1;
-        const int total_iters = ((num_tiles - int(blockIdx.x) + int(gridDim.x) - 1) /
-                                 int(gridDim.x)) * KB;
-        auto fetch = [&](int j, float &a_out, float (&b_out)[VB]) {
-            if (j >= total_iters)
-                return;
-            const int i = j / KB, kb = j - i * KB;
-            int tm, tn;
-            tile_coords(int(blockIdx.x) + i * int(gridDim.x), tiles_m, tiles_n, tm, tn);
-            a_out = __ldg(sa + size_t(kb) * M + tm * BM + row_in_tile);
-            const int ncol = tn * BN + col0;
-            if (MODE == 0) {
-                b_out[0] = __ldg(sb + size_t(ncol / 128) * KB + kb);
-            } else if (MODE == 1) {
-                b_out[0] = __ldg(sb + size_t(kb) * (N / 128) + ncol / 128);
-            } else {
-                const float *p = sb + size_t(kb) * N + ncol + lane * VB;
-#pragma unroll
-                for (int v = 0; v < VB; ++v)
-                    b_out[v] = __ldg(p + v);
-            }
-        };
-        float a0 = 0.f, a1 = 0.f, a2 = 0.f;
-        float b0[VB], b1[VB], b2[VB];
-#pragma unroll
-        for (int v = 0; v < VB; ++v)
-            b0[v] = b1[v] = b2[v] = 0.f;
-        fetch(0, a0, b0);
-        fetch(1, a1, b1);
+        const int my_tiles = (num_tiles - unit + units - 1) / units;
+        const int total_iters = my_tiles > 0 ? my_tiles * KB : 0;
 
-        int buf = 0;
+        int buf = 0, kb = 0, t = unit, tm = 0, tn = 0;
         uint32_t tphase = 0;
+        tile_coords(t, tiles_m, tiles_n, tm, tn);
         for (int j = 0; j < total_iters; ++j) {
-            fetch(j + 2, a2, b2);
-            const int i = j / KB, kb = j - i * KB;
-            if (MODE == 2) {
-#pragma unroll
-                for (int v = 0; v < VB; ++v)
-                    my_sbv[lane * VB + v] = b0[v];
-                __syncwarp();
-            }
-            const bool ready = mbar_wait_bounded(&tfull[buf], tphase, abort_flag,
-                                                 &g_device_error, ERR_EPI, WAIT_LIMIT_NS);
+            const int r = j % Cfg::SRING;
+            const bool sready = mbar_wait_bounded(&sfull[r], uint32_t(j / Cfg::SRING) & 1u,
+                                                  abort_flag, &g_device_error, ERR_SCALES,
+                                                  WAIT_LIMIT_NS);
+            const float *slot = sring + r * Cfg::SLOT_FLOATS;
+            const bool ready = sready && mbar_wait_bounded(&tfull[buf], tphase, abort_flag,
+                                                           &g_device_error, ERR_EPI,
+                                                           WAIT_LIMIT_NS);
             if (!__all_sync(0xffffffffu, ready))  // leave together: tcgen05.ld is warp-wide
                 break;
             tc_fence_after();
+            const float a_s = slot[row_local];
             const uint32_t taddr =
                 tmem_base + (uint32_t(quarter * 32) << 16) + uint32_t(buf * BN + col0);
-            const float sc = a0 * b0[0];
+            const float sc = (MODE == 2) ? a_s : a_s * slot[BM + col0 / 128];
             const float2 sc2 = make_float2(sc, sc);
-            const float2 sa2 = make_float2(a0, a0);
+
+            // TMEM -> registers in 32-column chunks; with 64 columns per thread both
+            // chunks are loaded before one wait.  The buffer goes back to the MMA as
+            // soon as the last chunk is in registers.
             constexpr int CHUNKS = COLS / 32;
-            constexpr int GROUP = 1;  // TMEM loads in flight per wait
-            static_assert(CHUNKS % GROUP == 0, "chunk grouping");
+            constexpr int GRP = (CHUNKS <= 2) ? CHUNKS : 1;
 #pragma unroll
-            for (int cg = 0; cg < CHUNKS; cg += GROUP) {
-                uint32_t v[GROUP][32];
+            for (int cg = 0; cg < CHUNKS; cg += GRP) {
+                uint32_t v[GRP][32];
 #pragma unroll
-                for (int g = 0; g < GROUP; ++g)
+                for (int g = 0; g < GRP; ++g)
                     tmem_ld_32x32b_x32(taddr + uint32_t((cg + g) * 32), v[g]);
                 tmem_wait_ld();
-                if (cg + GROUP == CHUNKS) {
-                    // Partial fully in registers: hand the TMEM buffer back to the MMA.
+                if (cg + GRP == CHUNKS) {
                     tc_fence_before();
                     __syncwarp();
-                    if (lane == 0)
-                        mbar_arrive(&tempty[buf]);
+                    if (lane == 0) {
+                        if (CG == 1 || rank == 0)
+                            mbar_arrive(&tempty[buf]);
+                        else  // the MMA issuer lives in the even CTA
+                            mbar_arrive_cluster(tempty_lead + uint32_t(buf) * 8u);
+                    }
                 }
 #pragma unroll
-                for (int g = 0; g < GROUP; ++g) {
+                for (int g = 0; g < GRP; ++g) {
                     const int c = cg + g;
 #pragma unroll
-                    for (int jj = 0; jj < 16; ++jj) {
-                        const float2 p = make_float2(__uint_as_float(v[g][2 * jj]),
-                                                     __uint_as_float(v[g][2 * jj + 1]));
+                    for (int jj = 0; jj < 16; jj += 2) {
+                        const float2 p0 = make_float2(__uint_as_float(v[g][2 * jj]),
+                                                      __uint_as_float(v[g][2 * jj + 1]));
+                        const float2 p1 = make_float2(__uint_as_float(v[g][2 * jj + 2]),
+                                                      __uint_as_float(v[g][2 * jj + 3]));
+                        float2 &a0 = acc[c * 16 + jj];
+                        float2 &a1 = acc[c * 16 + jj + 1];
                         if (MODE == 2) {
-                            const float2 bs = *reinterpret_cast<const float2 *>(
-                                my_sbv + c * 32 + 2 * jj);
-                            acc[c * 16 + jj] =
-                                __ffma2_rn(__fmul2_rn(p, bs), sa2, acc[c * 16 + jj]);
+                            const float4 bs = *reinterpret_cast<const float4 *>(
+                                slot + BM + col0 + c * 32 + 2 * jj);
+                            a0 = __ffma2_rn(__fmul2_rn(p0, make_float2(bs.x, bs.y)), sc2, a0);
+                            a1 = __ffma2_rn(__fmul2_rn(p1, make_float2(bs.z, bs.w)), sc2, a1);
                         } else {
-                            acc[c * 16 + jj] = __ffma2_rn(p, sc2, acc[c * 16 + jj]);
+                            a0 = __ffma2_rn(p0, sc2, a0);
+                            a1 = __ffma2_rn(p1, sc2, a1);
                         }
                     }
                 }
             }
-            if (MODE == 2)
-                __syncwarp();  // all lanes done reading my_sbv before it is rewritten
-            if (kb == KB - 1) {
-                int tm, tn;
-                tile_coords(int(blockIdx.x) + i * int(gridDim.x), tiles_m, tiles_n, tm, tn);
-                __nv_bfloat16 *dst =
-                    D + size_t(tm * BM + row_in_tile) * size_t(N) + size_t(tn * BN + col0);
+            __syncwarp();
+            if (lane == 0)
+                mbar_arrive(&sempty[r]);  // this warp is done with the slot's scales
+            if (++kb == KB) {
+                if (Cfg::TMA_STORE) {
+                    // BF16 tile -> swizzled staging -> two bulk tensor stores per warp.
+                    uint8_t *stg = sout + ew * Cfg::STAGE_OUT_WARP;
+                    if (lane == 0)
+                        bulk_wait_read0();  // the previous tile's stores have read it
+                    __syncwarp();
 #pragma unroll
-                for (int c = 0; c < COLS / 8; ++c) {
-                    uint4 o;
-                    __nv_bfloat162 h0 = __float22bfloat162_rn(acc[4 * c + 0]);
-                    __nv_bfloat162 h1 = __float22bfloat162_rn(acc[4 * c + 1]);
-                    __nv_bfloat162 h2 = __float22bfloat162_rn(acc[4 * c + 2]);
-                    __nv_bfloat162 h3 = __float22bfloat162_rn(acc[4 * c + 3]);
-                    o.x = *reinterpret_cast<uint32_t *>(&h0);
-                    o.y = *reinterpret_cast<uint32_t *>(&h1);
-                    o.z = *reinterpret_cast<uint32_t *>(&h2);
-                    o.w = *reinterpret_cast<uint32_t *>(&h3);
-                    *reinterpret_cast<uint4 *>(dst + c * 8) = o;
+                    for (int c = 0; c < COLS / 8; ++c) {
+                        uint4 o;
+                        __nv_bfloat162 h0 = __float22bfloat162_rn(acc[4 * c + 0]);
+                        __nv_bfloat162 h1 = __float22bfloat162_rn(acc[4 * c + 1]);
+                        __nv_bfloat162 h2 = __float22bfloat162_rn(acc[4 * c + 2]);
+                        __nv_bfloat162 h3 = __float22bfloat162_rn(acc[4 * c + 3]);
+                        o.x = *reinterpret_cast<uint32_t *>(&h0);
+                        o.y = *reinterpret_cast<uint32_t *>(&h1);
+                        o.z = *reinterpret_cast<uint32_t *>(&h2);
+                        o.w = *reinterpret_cast<uint32_t *>(&h3);
+                        const int box = c >> 3, chunk = c & 7;
+                        *reinterpret_cast<uint4 *>(stg + box * 4096 + lane * 128 +
+                                                   ((chunk ^ (lane & 7)) << 4)) = o;
+                    }
+                    fence_proxy_async_smem();
+                    __syncwarp();
+                    if (lane == 0) {
+                        const int r0 = tm * Cfg::TILE_M + rank * BM + quarter * 32;
+#pragma unroll
+                        for (int box = 0; box < COLS / 64; ++box)
+                            tma_store_2d(&tmD, stg + box * 4096, tn * BN + col0 + box * 64, r0);
+                        bulk_commit();
+                    }
+                } else {
+                    __nv_bfloat16 *dst = D + size_t(tm * Cfg::TILE_M + row_in_tile) * size_t(N) +
+                                         size_t(tn * BN + col0);
+#pragma unroll
+                    for (int c = 0; c < COLS / 8; ++c) {
+                        uint4 o;
+                        __nv_bfloat162 h0 = __float22bfloat162_rn(acc[4 * c + 0]);
+                        __nv_bfloat162 h1 = __float22bfloat162_rn(acc[4 * c + 1]);
+                        __nv_bfloat162 h2 = __float22bfloat162_rn(acc[4 * c + 2]);
+                        __nv_bfloat162 h3 = __float22bfloat162_rn(acc[4 * c + 3]);
+                        o.x = *reinterpret_cast<uint32_t *>(&h0);
+                        o.y = *reinterpret_cast<uint32_t *>(&h1);
+                        o.z = *reinterpret_cast<uint32_t *>(&h2);
+                        o.w = *reinterpret_cast<uint32_t *>(&h3);
+                        *reinterpret_cast<uint4 *>(dst + c * 8) = o;
+                    }
                 }
 #pragma unroll
                 for (int q = 0; q < COLS / 2; ++q)
                     acc[q] = make_float2(0.f, 0.f);
+                kb = 0;
+                t += units;
+                if (t < num_tiles)
+                    tile_coords(t, tiles_m, tiles_n, tm, tn);
             }
-            a0 = a1;
-            a1 = a2;
-#pragma unroll
-            for (int v = 0; v < VB; ++v) {
-                b0[v] = b1[v];
-                b1[v] = b2[v];
-            }
-            if (++buf == 2) {
+            if (++buf == Cfg::NBUF) {
                 buf = 0;
                 tphase ^= 1u;
             }
         }
+        if (Cfg::TMA_STORE && lane == 0)
+            bulk_wait0();  // output stores complete before the CTA leaves
     }
 
     tc_fence_before();
     __syncthreads();
-    if (*abort_flag) {
-        // Unwind: let every load and MMA still in flight land before the block's
-        // shared memory and tensor memory are released.
-        if (warp == 0 && lane == 0) {
-            for (int s = 0; s < STAGES; ++s)
-                if (armed_mask & (1u << s))
-                    mbar_wait_bounded(&full[s], (armed_parity >> s) & 1u, abort_flag,
-                                      &g_device_error, ERR_DRAIN, DRAIN_LIMIT_NS);
+    if (*abort_flag && threadIdx.x == 0) {
+        // Unwind after a wait ran out: give copies and MMAs still in flight time to
+        // land before the CTA's shared and tensor memory are released.
+        const uint64_t t0 = global_timer_ns();
+        while (global_timer_ns() - t0 < DRAIN_NS) {
         }
-        if (warp == 1 && lane == 0 && last_buf >= 0) {
-            // The flag is already set, so poll directly with a time limit.
-            uint64_t t0 = global_timer_ns();
-            while (!mbar_try_wait(&tfull[last_buf], last_tparity) &&
-                   global_timer_ns() - t0 < DRAIN_LIMIT_NS) {
-            }
-        }
-        __syncthreads();
     }
+    if (CG == 2)
+        cluster_sync();  // the partner no longer reads this CTA's memory or barriers
+    else
+        __syncthreads();
     if (warp == 1) {
         tc_fence_after();
-        tmem_dealloc(tmem_base, Cfg::TMEM_COLS);
+        tmem_dealloc<CG>(tmem_base, Cfg::TMEM_COLS);
     }
 }
 
@@ -412,10 +519,10 @@ static EncodeTiledFn get_encode_fn()
     return fn;
 }
 
-// 2-D uint8 tensor map over a row-major [rows][cols] array, box {box_cols, box_rows},
-// 128-byte swizzle.
+// 2-D uint8 tensor map over a row-major [rows][cols] array, box {box_cols, box_rows}.
 static bool make_map_u8(CUtensorMap *map, const void *base, uint64_t rows, uint64_t cols,
-                        uint32_t box_rows, uint32_t box_cols)
+                        uint32_t box_rows, uint32_t box_cols,
+                        CUtensorMapSwizzle swz = CU_TENSOR_MAP_SWIZZLE_128B)
 {
     EncodeTiledFn enc = get_encode_fn();
     if (!enc)
@@ -425,8 +532,25 @@ static bool make_map_u8(CUtensorMap *map, const void *base, uint64_t rows, uint6
     cuuint32_t box[2] = {box_cols, box_rows};
     cuuint32_t estride[2] = {1, 1};
     CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void *>(base), gdim, gstride,
-                     box, estride, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                     box, estride, CU_TENSOR_MAP_INTERLEAVE_NONE, swz,
                      CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS;
+}
+
+// BF16 [rows][cols] output map for TMA stores: box 64 columns (128 B) x 32 rows,
+// 128-byte swizzle.
+static bool make_map_bf16_out(CUtensorMap *map, void *base, uint64_t rows, uint64_t cols)
+{
+    EncodeTiledFn enc = get_encode_fn();
+    if (!enc)
+        return false;
+    cuuint64_t gdim[2] = {cols, rows};
+    cuuint64_t gstride[1] = {cols * 2};
+    cuuint32_t box[2] = {64, 32};
+    cuuint32_t estride[2] = {1, 1};
+    CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, base, gdim, gstride, box, estride,
+                     CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                     CU_TENSOR_MAP_L2_PROMOTION_NONE, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     return r == CUDA_SUCCESS;
 }
 
@@ -451,33 +575,82 @@ static cudaError_t run(const uint8_t *a, const float *sa, const uint8_t *b, cons
         return cudaErrorInvalidValue;
     bool ok;
     if (Cfg::MODE == 1)
-        ok = make_map_u8(&tb, b, uint64_t(K), uint64_t(N), BK, 128);  // W[K][N], N contiguous
+        ok = make_map_u8(&tb, b, uint64_t(K), uint64_t(N), BK, Cfg::B_BOX,  // W[K][N]
+                         Cfg::B_BOX == 128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B);
     else
-        ok = make_map_u8(&tb, b, uint64_t(N), uint64_t(K), Cfg::BN, BK);
+        ok = make_map_u8(&tb, b, uint64_t(N), uint64_t(K), Cfg::B_ROWS, BK);
     if (!ok)
         return cudaErrorInvalidValue;
-    const int64_t tiles = (M / BM) * (N / Cfg::BN);
-    const int grid = int(tiles < num_sms ? tiles : num_sms);
-    fp8_gemm_kernel<Cfg><<<grid, Cfg::THREADS, Cfg::SMEM, stream>>>(
-        ta, tb, sa, sb, static_cast<__nv_bfloat16 *>(d), int(M), int(N), int(K));
+    CUtensorMap td;
+    std::memset(&td, 0, sizeof td);
+    if (Cfg::TMA_STORE && !make_map_bf16_out(&td, d, uint64_t(M), uint64_t(N)))
+        return cudaErrorInvalidValue;
+    const int64_t tiles = (M / Cfg::TILE_M) * (N / Cfg::BN);
+    __nv_bfloat16 *dp = static_cast<__nv_bfloat16 *>(d);
+    if (Cfg::CG == 1) {
+        const int grid = int(tiles < num_sms ? tiles : num_sms);
+        kern<<<grid, Cfg::THREADS, Cfg::SMEM, stream>>>(ta, tb, td, sa, sb, dp, int(M), int(N),
+                                                         int(K));
+        return cudaGetLastError();
+    }
+    cudaLaunchConfig_t cfg = {};
+    cudaLaunchAttribute at[1];
+    at[0].id = cudaLaunchAttributeClusterDimension;
+    at[0].val.clusterDim.x = 2;
+    at[0].val.clusterDim.y = 1;
+    at[0].val.clusterDim.z = 1;
+    cfg.blockDim = dim3(Cfg::THREADS);
+    cfg.dynamicSmemBytes = Cfg::SMEM;
+    cfg.stream = stream;
+    cfg.attrs = at;
+    cfg.numAttrs = 1;
+    cfg.gridDim = dim3(2 * unsigned(num_sms / 2));
+    int max_clusters = 0;
+    e = cudaOccupancyMaxActiveClusters(&max_clusters, kern, &cfg);
+    if (e != cudaSuccess)
+        return e;
+    if (max_clusters < 1)
+        return cudaErrorInvalidConfiguration;
+    const int64_t clusters = tiles < max_clusters ? tiles : max_clusters;
+    cfg.gridDim = dim3(unsigned(2 * clusters));
+    e = cudaLaunchKernelEx(&cfg, kern, ta, tb, td, sa, sb, dp, int(M), int(N), int(K));
+    if (e != cudaSuccess)
+        return e;
     return cudaGetLastError();
 }
+
+#ifndef FP8BW_PAIR
+#define FP8BW_PAIR 1
+#endif
+#ifndef FP8BW_PAIR_BN
+#define FP8BW_PAIR_BN 256
+#endif
 
 cudaError_t launch_gemm(int mode, const uint8_t *a, const float *sa, const uint8_t *b,
                         const float *sb, void *d, int64_t M, int64_t N, int64_t K,
                         cudaStream_t stream, int num_sms)
 {
+    constexpr int PBN = FP8BW_PAIR_BN;                 // N of a pair tile
+    constexpr int PST = (PBN == 256) ? 4 : 6;          // pair-path pipeline stages
     const bool wide = (N % 256) == 0;
+    const bool pair = FP8BW_PAIR && (N % PBN) == 0 && (M % 256) == 0 &&
+                      (M / 256) * (N / PBN) >= 16;
     switch (mode) {
     case 0:
-        return wide ? run<GemmCfg<256, 0, 4>>(a, sa, b, sb, d, M, N, K, stream, num_sms)
-                    : run<GemmCfg<128, 0, 6>>(a, sa, b, sb, d, M, N, K, stream, num_sms);
+        if (pair)
+            return run<GemmCfg<PBN, 0, PST, 2>>(a, sa, b, sb, d, M, N, K, stream, num_sms);
+        return wide ? run<GemmCfg<256, 0, 4, 1>>(a, sa, b, sb, d, M, N, K, stream, num_sms)
+                    : run<GemmCfg<128, 0, 6, 1>>(a, sa, b, sb, d, M, N, K, stream, num_sms);
     case 1:
-        return wide ? run<GemmCfg<256, 1, 4>>(a, sa, b, sb, d, M, N, K, stream, num_sms)
-                    : run<GemmCfg<128, 1, 6>>(a, sa, b, sb, d, M, N, K, stream, num_sms);
+        if (pair)
+            return run<GemmCfg<PBN, 1, PST, 2>>(a, sa, b, sb, d, M, N, K, stream, num_sms);
+        return wide ? run<GemmCfg<256, 1, 4, 1>>(a, sa, b, sb, d, M, N, K, stream, num_sms)
+                    : run<GemmCfg<128, 1, 6, 1>>(a, sa, b, sb, d, M, N, K, stream, num_sms);
     default:
-        return wide ? run<GemmCfg<256, 2, 4>>(a, sa, b, sb, d, M, N, K, stream, num_sms)
-                    : run<GemmCfg<128, 2, 6>>(a, sa, b, sb, d, M, N, K, stream, num_sms);
+        if (pair)
+            return run<GemmCfg<PBN, 2, PST, 2>>(a, sa, b, sb, d, M, N, K, stream, num_sms);
+        return wide ? run<GemmCfg<256, 2, 4, 1>>(a, sa, b, sb, d, M, N, K, stream, num_sms)
+                    : run<GemmCfg<128, 2, 6, 1>>(a, sa, b, sb, d, M, N, K, stream, num_sms);
     }
 }
 

@@ -85,9 +85,10 @@ __device__ __forceinline__ uint2 quant8(uint4 v, const GroupDiv &div)
 
 // ------------------------------------------------------------ fp8_quant_act
 
-// A warp quantizes two groups at a time: half-warp h takes group (kb, m + h); each
-// lane holds 8 consecutive values (16 bytes).  Groups are enumerated g = kb*M + m
-// so the scale writes of neighbouring warps are contiguous.
+// A warp quantizes two consecutive groups at a time (half-warp h takes group
+// 2p + h); each lane holds 8 consecutive values (16 bytes).  Groups are enumerated
+// in memory order, g = m*(K/128) + kb, so the warps in flight stream through one
+// contiguous region of X and Q; the scale of group (m, kb) goes to s[kb][m].
 constexpr int QA_THREADS = 256;
 constexpr int QA_UNROLL = 4;
 
@@ -109,9 +110,7 @@ quant_act_kernel(const uint4 *__restrict__ x, int64_t M, int64_t K, uint2 *__res
             int64_t p = p0 + int64_t(u) * nwarps;
             off[u] = -1;
             if (p < npairs) {
-                int64_t g = 2 * p + half;
-                int64_t kb = g / M, m = g - kb * M;
-                off[u] = (m * K + kb * 128) / 8 + sub;  // in units of 8 elements
+                off[u] = (2 * p + half) * 16 + sub;  // in units of 8 elements
                 v[u] = __ldg(x + off[u]);
             }
         }
@@ -130,8 +129,11 @@ quant_act_kernel(const uint4 *__restrict__ x, int64_t M, int64_t K, uint2 *__res
             if (amax != 0.0f)
                 codes = quant8(v[u], GroupDiv(sc));
             q[off[u]] = codes;
-            if (sub == 0)
-                s[2 * p + half] = sc;
+            if (sub == 0) {
+                const int64_t g = 2 * p + half, KB = K / 128;
+                const int64_t m = g / KB, kb = g - m * KB;
+                s[kb * M + m] = sc;
+            }
         }
     }
 }

@@ -20,6 +20,8 @@ BF16 tensors are returned as numpy ``uint16`` bit patterns.
 """
 from __future__ import annotations
 
+import os
+
 import numpy as np
 
 GOLDEN = np.uint64(0x9E3779B97F4A7C15)
@@ -92,12 +94,24 @@ def normal_bf16(rows: int, cols: int, std: float, seed: int,
     if outliers:
         gain = np.ones(cols, dtype=np.float64)
         gain[outlier_columns(seed, cols)] = outlier_gain
-    for s in range(0, total, _CHUNK):
+
+    def fill(s):
         n = min(_CHUNK, total - s)
         z = standard_normal(seed, n, start=s) * std
         if gain is not None:
             z *= gain[(np.arange(s, s + n) % cols)]
         out[s:s + n] = f64_to_bf16_bits(z)
+
+    starts = range(0, total, _CHUNK)
+    if total > 4 * _CHUNK:
+        # chunks are independent slices of the counter-based stream, so filling
+        # them on several threads gives the same bytes
+        from concurrent.futures import ThreadPoolExecutor
+        with ThreadPoolExecutor(max_workers=min(16, os.cpu_count() or 1)) as ex:
+            list(ex.map(fill, starts))
+    else:
+        for s in starts:
+            fill(s)
     return out.reshape(rows, cols)
 
 
