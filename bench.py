@@ -65,6 +65,31 @@ def dist_env():
     return world, rank, local
 
 
+def kernel_source_digest():
+    """SHA-256 over the GEMM kernel sources: ncu traffic figures are only reported
+    while the kernel they were taken on is unchanged."""
+    import hashlib
+    h = hashlib.sha256()
+    for f in ("gemm.cu", "ptx.cuh"):
+        with open(os.path.join(ROOT, "blockwise_fp8_linear_b200", "csrc", f), "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()
+
+
+def recorded_traffic():
+    """DRAM bytes per GEMM launch from the committed ncu summary, or None if the
+    summary is missing or was taken on different kernel sources."""
+    path = os.path.join(ROOT, "profiles", "gemm_dram_traffic_qwen3_block_m8192.json")
+    try:
+        with open(path) as f:
+            rec = json.load(f)
+    except (OSError, ValueError):
+        return None
+    if rec.get("gemm_source_sha256") != kernel_source_digest():
+        return None
+    return rec.get("dram_bytes_per_launch")
+
+
 def measured_peaks():
     path = os.path.join(ROOT, "MEASURED_PEAKS.json")
     try:
@@ -324,7 +349,8 @@ def run_ours(args):
         "bound": "tensor", "achieved": round(achieved, 2),
         "peak": round(fp8_peak, 1), "unit": "TFLOP/s", "frac": round(achieved / fp8_peak, 4),
         "peak_source": f"{peak_src} cuBLAS bf16 burst x {FP8_OVER_BF16:g} (nominal FP8:BF16)",
-        "traffic": None,
+        "traffic": recorded_traffic(),
+        "traffic_unit": "bytes per GEMM launch (mean over the step's 12 GEMMs, ncu dram read+write)",
         "gemm_share_of_step": round(gemm_ms / local_ms, 4),
     }
 

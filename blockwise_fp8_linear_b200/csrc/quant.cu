@@ -44,20 +44,20 @@ struct GroupDiv {
         fast = scale >= 0x1p-90f && scale <= 0x1p90f;
         r = fast ? __frcp_rn(scale) : 0.0f;
     }
-    __device__ __forceinline__ float operator()(float x) const
-    {
-        if (fast) {
-            float q0 = __fmul_rn(x, r);
-            float e = __fmaf_rn(-q0, s, x);
-            float q = __fmaf_rn(e, r, q0);
-            return copysignf(q, x);
-        }
-        return __fdiv_rn(x, s);
-    }
 };
 
 __device__ __forceinline__ float bf16lo(uint32_t w) { return __uint_as_float(w << 16); }
 __device__ __forceinline__ float bf16hi(uint32_t w) { return __uint_as_float(w & 0xFFFF0000u); }
+
+// Fast-path quotients of a pair of values by per-lane-half scales (s, r, -s given as
+// packed pairs): q0 = x*r, e = x - q0*s (one FMA, exact), q = q0 + e*r.
+__device__ __forceinline__ float2 div2_fast(float2 x, float2 r, float2 neg_s)
+{
+    const float2 q0 = __fmul2_rn(x, r);
+    const float2 e = __ffma2_rn(q0, neg_s, x);
+    const float2 q = __ffma2_rn(e, r, q0);
+    return make_float2(copysignf(q.x, x.x), copysignf(q.y, x.y));
+}
 
 // |bf16| max over two packed words, as packed unsigned 16-bit halves (for
 // non-negative BF16 values the integer order is the numeric order).
@@ -72,15 +72,24 @@ __device__ __forceinline__ float halves_max_to_float(uint32_t m2)
     return __uint_as_float(m << 16);
 }
 
-// Eight BF16 values (one uint4) -> eight E4M3 codes (one uint2).
-__device__ __forceinline__ uint2 quant8(uint4 v, const GroupDiv &div)
+// Eight BF16 values of one group (one uint4) -> eight E4M3 codes (one uint2).
+__device__ __forceinline__ uint2 quant8(uint4 v, const GroupDiv &d)
 {
-    uint2 o;
-    o.x = cvt_e4m3x2(div(bf16lo(v.x)), div(bf16hi(v.x))) |
-          (cvt_e4m3x2(div(bf16lo(v.y)), div(bf16hi(v.y))) << 16);
-    o.y = cvt_e4m3x2(div(bf16lo(v.z)), div(bf16hi(v.z))) |
-          (cvt_e4m3x2(div(bf16lo(v.w)), div(bf16hi(v.w))) << 16);
-    return o;
+    const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+    uint32_t c[4];
+    if (d.fast) {
+        const float2 r2 = make_float2(d.r, d.r), ns2 = make_float2(-d.s, -d.s);
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            const float2 q = div2_fast(make_float2(bf16lo(w[i]), bf16hi(w[i])), r2, ns2);
+            c[i] = cvt_e4m3x2(q.x, q.y);
+        }
+    } else {
+#pragma unroll
+        for (int i = 0; i < 4; ++i)
+            c[i] = cvt_e4m3x2(__fdiv_rn(bf16lo(w[i]), d.s), __fdiv_rn(bf16hi(w[i]), d.s));
+    }
+    return make_uint2(c[0] | (c[1] << 16), c[2] | (c[3] << 16));
 }
 
 // ------------------------------------------------------------ fp8_quant_act
@@ -131,7 +140,15 @@ quant_act_kernel(const uint4 *__restrict__ x, int64_t M, int64_t K, uint2 *__res
             q[off[u]] = codes;
             if (sub == 0) {
                 const int64_t g = 2 * p + half, KB = K / 128;
-                const int64_t m = g / KB, kb = g - m * KB;
+                int64_t m, kb;
+                if (g < INT32_MAX) {  // 32-bit division in the common case
+                    const uint32_t g32 = uint32_t(g), kb32 = uint32_t(KB);
+                    m = g32 / kb32;
+                    kb = g32 - uint32_t(m) * kb32;
+                } else {
+                    m = g / KB;
+                    kb = g - m * KB;
+                }
                 s[kb * M + m] = sc;
             }
         }
@@ -176,19 +193,32 @@ quant_act_t_kernel(const uint32_t *__restrict__ x, int64_t M, int64_t K,
     const float s_lo = __fdiv_rn(amax_lo, 448.0f);
     const float s_hi = __fdiv_rn(amax_hi, 448.0f);
 
+    // Lane values: v[r] holds (column 2l, column 2l+1) of row r, whose groups have
+    // the scales s_lo and s_hi, so each packed pair divides by a packed scale pair.
     uint32_t clo[4] = {0u, 0u, 0u, 0u}, chi[4] = {0u, 0u, 0u, 0u};
-    if (amax_lo != 0.0f) {
-        GroupDiv d(s_lo);
+    const GroupDiv dlo(s_lo), dhi(s_hi);
+    if (dlo.fast && dhi.fast) {
+        const float2 r2 = make_float2(dlo.r, dhi.r), ns2 = make_float2(-s_lo, -s_hi);
 #pragma unroll
-        for (int r = 0; r < 16; r += 2)
-            clo[r / 4] |= cvt_e4m3x2(d(bf16lo(v[r])), d(bf16lo(v[r + 1]))) << (16 * ((r / 2) & 1));
-    }
-    if (amax_hi != 0.0f) {
-        GroupDiv d(s_hi);
+        for (int r = 0; r < 16; r += 2) {
+            const float2 a = div2_fast(make_float2(bf16lo(v[r]), bf16hi(v[r])), r2, ns2);
+            const float2 b = div2_fast(make_float2(bf16lo(v[r + 1]), bf16hi(v[r + 1])), r2, ns2);
+            clo[r / 4] |= cvt_e4m3x2(a.x, b.x) << (16 * ((r / 2) & 1));
+            chi[r / 4] |= cvt_e4m3x2(a.y, b.y) << (16 * ((r / 2) & 1));
+        }
+    } else {
 #pragma unroll
-        for (int r = 0; r < 16; r += 2)
-            chi[r / 4] |= cvt_e4m3x2(d(bf16hi(v[r])), d(bf16hi(v[r + 1]))) << (16 * ((r / 2) & 1));
+        for (int r = 0; r < 16; r += 2) {
+            clo[r / 4] |= cvt_e4m3x2(__fdiv_rn(bf16lo(v[r]), s_lo), __fdiv_rn(bf16lo(v[r + 1]), s_lo))
+                          << (16 * ((r / 2) & 1));
+            chi[r / 4] |= cvt_e4m3x2(__fdiv_rn(bf16hi(v[r]), s_hi), __fdiv_rn(bf16hi(v[r + 1]), s_hi))
+                          << (16 * ((r / 2) & 1));
+        }
     }
+    if (amax_lo == 0.0f)
+        clo[0] = clo[1] = clo[2] = clo[3] = 0u;
+    if (amax_hi == 0.0f)
+        chi[0] = chi[1] = chi[2] = chi[3] = 0u;
     const int64_t col = k0 + 2 * l;
     *reinterpret_cast<uint4 *>(qt + col * M + row0) = make_uint4(clo[0], clo[1], clo[2], clo[3]);
     *reinterpret_cast<uint4 *>(qt + (col + 1) * M + row0) = make_uint4(chi[0], chi[1], chi[2], chi[3]);
