@@ -4,9 +4,10 @@
 One step = one pass of the whole hot path over the four linear layers of a
 Qwen3-1.7B transformer block at M = 8192 tokens (micro-batch 2 x sequence 4096):
 QKV (2048 -> 4096), O (2048 -> 2048), gate/up (2048 -> 12288), down (6144 -> 2048).
-For each linear: fp8_quant_act(X), fp8_quant_weight(W), fprop; fp8_quant_act(dY),
-dgrad; fp8_quant_act_t(dY), fp8_quant_act_t(X), wgrad -- 32 kernel launches, 2.47
-TFLOP of GEMM work.  The metric is TFLOP/s of the whole step (2MNK summed over the
+For each linear: fp8_quant_act_dual(X) (row-wise and token-wise copies from one read),
+fp8_quant_weight(W), fprop; fp8_quant_act_dual(dY), dgrad; wgrad -- 24 kernel
+launches, 2.47 TFLOP of GEMM work (--separate-quant: the four single-layout passes,
+32 launches).  The metric is TFLOP/s of the whole step (2MNK summed over the
 12 GEMMs, divided by the time of all quantizers and GEMMs).
 
 Inputs are seeded synthetic BF16 tensors (X ~ N(0,1) with 1% outlier channels x20,
@@ -40,7 +41,6 @@ TOKENS = 8192
 LINEARS = [("qkv", 2048, 4096), ("o", 2048, 2048), ("gate_up", 2048, 12288), ("down", 6144, 2048)]
 WORKLOAD = "qwen3-1.7b block linears (qkv, o, gate_up, down) fprop+dgrad+wgrad, M=8192"
 STEP_FLOPS = sum(3 * 2 * TOKENS * din * dout for _, din, dout in LINEARS)
-LAUNCHES_PER_STEP = 8 * len(LINEARS)
 FP8_OVER_BF16 = 4.5 / 2.25  # nominal dense FP8 : BF16 tensor throughput on B200
 
 
@@ -49,7 +49,7 @@ def config_dict(n):
         "workload": WORKLOAD,
         "tokens": TOKENS,
         "linears": {name: [din, dout] for name, din, dout in LINEARS},
-        "passes": "fprop+dgrad+wgrad with all quantizers",
+        "passes": "fprop+dgrad+wgrad with all quantizers (X and dY quantized once into both layouts)",
         "step_gflop": round(STEP_FLOPS / 1e9, 3),
         "l2": "inputs larger than L2 (637 MB of BF16 inputs per step), no flush",
         "parallelism": f"replicas x{n}" if n > 1 else "single GPU",
@@ -159,11 +159,13 @@ class ClockSampler:
 class LayerWork:
     """Device buffers of one step and the launch sequence through the C ABI."""
 
-    def __init__(self, dev, host_inputs):
+    def __init__(self, dev, host_inputs, separate=False):
         import torch
         import blockwise_fp8_linear_b200 as fb
         self.fb = fb
         self.torch = torch
+        self.separate = separate
+        self.launches_per_step = (8 if separate else 6) * len(LINEARS)
         self.lin = []
         for (name, din, dout), (X, W, dY) in zip(LINEARS, host_inputs):
             t = lambda a: torch.from_numpy(a.view(np.int16)).view(torch.bfloat16)
@@ -215,14 +217,23 @@ class LayerWork:
 
         for d in self.lin:
             din, dout = d["din"], d["dout"]
-            chk(L.fp8_quant_act(d["X"].data_ptr(), T, din, d["qx"].data_ptr(), d["sx"].data_ptr(), st), "qa")
+            if self.separate:
+                chk(L.fp8_quant_act(d["X"].data_ptr(), T, din, d["qx"].data_ptr(), d["sx"].data_ptr(), st), "qa")
+            else:  # X read once: row-wise copy for fprop, token-wise copy kept for wgrad
+                chk(L.fp8_quant_act_dual(d["X"].data_ptr(), T, din, d["qx"].data_ptr(), d["sx"].data_ptr(),
+                                         d["qxt"].data_ptr(), d["sxt"].data_ptr(), st), "qd")
             chk(L.fp8_quant_weight(d["W"].data_ptr(), dout, din, d["qw"].data_ptr(),
                                    d["sw"].data_ptr(), None, st), "qw")
             gemm(fb.FPROP, d["qx"], d["sx"], d["qw"], d["sw"], d["Y"], T, dout, din)
-            chk(L.fp8_quant_act(d["dY"].data_ptr(), T, dout, d["qdy"].data_ptr(), d["sdy"].data_ptr(), st), "qa")
+            if self.separate:
+                chk(L.fp8_quant_act(d["dY"].data_ptr(), T, dout, d["qdy"].data_ptr(), d["sdy"].data_ptr(), st), "qa")
+            else:
+                chk(L.fp8_quant_act_dual(d["dY"].data_ptr(), T, dout, d["qdy"].data_ptr(), d["sdy"].data_ptr(),
+                                         d["qdyt"].data_ptr(), d["sdyt"].data_ptr(), st), "qd")
             gemm(fb.DGRAD, d["qdy"], d["sdy"], d["qw"], d["sw"], d["dX"], T, din, dout)
-            chk(L.fp8_quant_act_t(d["dY"].data_ptr(), T, dout, d["qdyt"].data_ptr(), d["sdyt"].data_ptr(), st), "qt")
-            chk(L.fp8_quant_act_t(d["X"].data_ptr(), T, din, d["qxt"].data_ptr(), d["sxt"].data_ptr(), st), "qt")
+            if self.separate:
+                chk(L.fp8_quant_act_t(d["dY"].data_ptr(), T, dout, d["qdyt"].data_ptr(), d["sdyt"].data_ptr(), st), "qt")
+                chk(L.fp8_quant_act_t(d["X"].data_ptr(), T, din, d["qxt"].data_ptr(), d["sxt"].data_ptr(), st), "qt")
             gemm(fb.WGRAD, d["qdyt"], d["sdyt"], d["qxt"], d["sxt"], d["dW"], dout, din, T)
 
 
@@ -269,7 +280,7 @@ def run_ours(args):
     import blockwise_fp8_linear_b200 as fb
 
     host = make_inputs(rank)
-    work = LayerWork(dev, host)
+    work = LayerWork(dev, host, separate=args.separate_quant)
 
     # warm-up
     for _ in range(args.warmup):
@@ -365,7 +376,7 @@ def run_ours(args):
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
             "dtype": "e4m3", "data": "synthetic (seeded splitmix64/Box-Muller BF16)",
             "config": config_dict(world), "roofline": roofline, "cpu_baseline": cpu,
-            "e2e": e2e, "gpu_launches": LAUNCHES_PER_STEP * args.steps,
+            "e2e": e2e, "gpu_launches": work.launches_per_step * args.steps,
             "clocks": clock_info,
             "pct_of_fp8_peak": round(100 * value / world / fp8_peak, 2),
         }
@@ -528,6 +539,9 @@ def main():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu", action="store_true")
     ap.add_argument("--cpu-budget", type=float, default=15.0, help="seconds of oracle work")
+    ap.add_argument("--separate-quant", action="store_true",
+                    help="quantize X and dY with separate row-wise and token-wise passes "
+                         "instead of the fused dual-output quantizer")
     ap.add_argument("--kernel-only", choices=KERNEL_CASES, default=None,
                     help="launch one kernel repeatedly (for profilers); no JSON metric line")
     args = ap.parse_args()

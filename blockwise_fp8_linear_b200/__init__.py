@@ -19,7 +19,8 @@ import os
 
 __all__ = [
     "FPROP", "DGRAD", "WGRAD", "Fp8bwError", "lib", "library_path",
-    "fp8_quant_act", "fp8_quant_act_t", "fp8_quant_weight", "fp8_gemm_blockwise",
+    "fp8_quant_act", "fp8_quant_act_t", "fp8_quant_act_dual", "fp8_quant_weight",
+    "fp8_gemm_blockwise",
     "fp8bw_status_string", "fp8bw_last_device_error", "fp8bw_version",
     "linear_fprop", "linear_dgrad", "linear_wgrad",
 ]
@@ -49,9 +50,11 @@ def lib():
         vp, i64, i32 = C.c_void_p, C.c_int64, C.c_int
         L.fp8_quant_act.argtypes = [vp, i64, i64, vp, vp, vp]
         L.fp8_quant_act_t.argtypes = [vp, i64, i64, vp, vp, vp]
+        L.fp8_quant_act_dual.argtypes = [vp, i64, i64, vp, vp, vp, vp, vp]
         L.fp8_quant_weight.argtypes = [vp, i64, i64, vp, vp, vp, vp]
         L.fp8_gemm_blockwise.argtypes = [i32, vp, vp, vp, vp, vp, i64, i64, i64, vp]
-        for f in (L.fp8_quant_act, L.fp8_quant_act_t, L.fp8_quant_weight, L.fp8_gemm_blockwise):
+        for f in (L.fp8_quant_act, L.fp8_quant_act_t, L.fp8_quant_act_dual, L.fp8_quant_weight,
+                  L.fp8_gemm_blockwise):
             f.restype = i32
         L.fp8bw_status_string.argtypes = [i32]
         L.fp8bw_status_string.restype = C.c_char_p
@@ -120,6 +123,20 @@ def fp8_quant_act_t(x, qt=None, st=None, stream=None):
     _check(lib().fp8_quant_act_t(x.data_ptr(), M, K, qt.data_ptr(), st.data_ptr(),
                                  _stream(stream)), "fp8_quant_act_t")
     return qt, st
+
+
+def fp8_quant_act_dual(x, q=None, s=None, qt=None, st=None, stream=None):
+    """X[M][K] bf16 -> (Q, S, Q^T, S^T): both layouts from one read of X."""
+    import torch
+    _need(x, torch.bfloat16, 2, "x")
+    M, K = x.shape
+    q = torch.empty((M, K), dtype=torch.uint8, device=x.device) if q is None else q
+    s = torch.empty((K // 128, M), dtype=torch.float32, device=x.device) if s is None else s
+    qt = torch.empty((K, M), dtype=torch.uint8, device=x.device) if qt is None else qt
+    st = torch.empty((M // 128, K), dtype=torch.float32, device=x.device) if st is None else st
+    _check(lib().fp8_quant_act_dual(x.data_ptr(), M, K, q.data_ptr(), s.data_ptr(), qt.data_ptr(),
+                                    st.data_ptr(), _stream(stream)), "fp8_quant_act_dual")
+    return q, s, qt, st
 
 
 def fp8_quant_weight(w, want_t: bool = False, q=None, s=None, qt=None, stream=None):

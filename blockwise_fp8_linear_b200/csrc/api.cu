@@ -126,6 +126,22 @@ int fp8_quant_act_t(const void *x_bf16, int64_t M, int64_t K, uint8_t *qt, float
         fp8bw::launch_quant_act_t(x_bf16, M, K, qt, st_, static_cast<cudaStream_t>(stream)));
 }
 
+int fp8_quant_act_dual(const void *x_bf16, int64_t M, int64_t K, uint8_t *q, float *s,
+                       uint8_t *qt, float *st_, void *stream)
+{
+    if (!x_bf16 || !q || !s || !qt || !st_)
+        return FP8BW_EINVAL;
+    if (!dim_ok(M) || !dim_ok(K))
+        return FP8BW_ESHAPE;
+    if (!aligned16(x_bf16) || !aligned16(q) || !aligned16(s) || !aligned16(qt) || !aligned16(st_))
+        return FP8BW_EALIGN;
+    int st;
+    if (device_sms({x_bf16, q, s, qt, st_}, &st) < 0)
+        return st;
+    return from_cuda(fp8bw::launch_quant_dual(x_bf16, M, K, q, s, qt, st_,
+                                              static_cast<cudaStream_t>(stream)));
+}
+
 int fp8_quant_weight(const void *w_bf16, int64_t N, int64_t K, uint8_t *q, float *s,
                      uint8_t *qt_or_null, void *stream)
 {

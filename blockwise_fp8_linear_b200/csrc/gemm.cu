@@ -242,10 +242,10 @@ fp8_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__
             uint32_t phase = 0, tphase = 0;
             for (int t = unit; t < num_tiles && !*abort_flag; t += units) {
                 for (int kb = 0; kb < KB; ++kb) {
-                    if (!mbar_wait_bounded(&full[stage], phase, abort_flag, &g_device_error,
+                    if (!mbar_spin_bounded(&full[stage], phase, abort_flag, &g_device_error,
                                            ERR_MMA_FULL, WAIT_LIMIT_NS))
                         goto role_done;
-                    if (!mbar_wait_bounded(&tempty[buf], tphase ^ 1u, abort_flag, &g_device_error,
+                    if (!mbar_spin_bounded(&tempty[buf], tphase ^ 1u, abort_flag, &g_device_error,
                                            ERR_MMA_TEMPTY, WAIT_LIMIT_NS))
                         goto role_done;
                     tc_fence_after();
@@ -354,7 +354,8 @@ fp8_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__
                                                   abort_flag, &g_device_error, ERR_SCALES,
                                                   WAIT_LIMIT_NS);
             const float *slot = sring + r * Cfg::SLOT_FLOATS;
-            const bool ready = sready && mbar_wait_bounded(&tfull[buf], tphase, abort_flag,
+            // busy-poll: this handshake is on the critical path of every block
+            const bool ready = sready && mbar_spin_bounded(&tfull[buf], tphase, abort_flag,
                                                            &g_device_error, ERR_EPI,
                                                            WAIT_LIMIT_NS);
             if (!__all_sync(0xffffffffu, ready))  // leave together: tcgen05.ld is warp-wide

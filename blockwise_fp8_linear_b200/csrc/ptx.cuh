@@ -80,6 +80,44 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t *bar, uint32_t parity)
     return ok != 0;
 }
 
+// Non-blocking test of the phase with `parity`.
+__device__ __forceinline__ bool mbar_test_wait(uint64_t *bar, uint32_t parity)
+{
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.test_wait.parity.acquire.cta.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(smem_u32(bar)), "r"(parity)
+        : "memory");
+    return ok != 0;
+}
+
+// Busy-polling version of mbar_wait_bounded (no suspension between tests), for the
+// latency-critical handshakes between the MMA warp and the epilogue.
+__device__ __forceinline__ bool mbar_spin_bounded(uint64_t *bar, uint32_t parity,
+                                                  volatile int *abort, int *err, int code,
+                                                  uint64_t limit_ns)
+{
+    if (mbar_test_wait(bar, parity))
+        return true;
+    uint64_t t0 = global_timer_ns();
+    for (uint32_t it = 1;; ++it) {
+        if (mbar_test_wait(bar, parity))
+            return true;
+        if ((it & 255u) == 0) {
+            if (*abort)
+                return false;
+            if (global_timer_ns() - t0 > limit_ns) {
+                atomicCAS(err, 0, code);
+                *abort = 1;
+                return false;
+            }
+        }
+    }
+}
+
 // A wait that gives up: polls the barrier until the phase with `parity` completes,
 // `*abort` becomes nonzero, or `limit_ns` of wall time pass.  On running out it
 // records `code` in the device error word and raises the block's abort flag.

@@ -297,11 +297,140 @@ quant_weight_kernel(const uint4 *__restrict__ w, int64_t N, int64_t K, uint2 *__
     }
 }
 
+// ------------------------------------------------------- tile quantizer (dual)
+
+// One CTA per 128 x 128 tile of X (one reduction block of 128 rows).  Every thread
+// first loads its 8 x 16 bytes (rows t/16 + 16p, columns 8*(t%16) .. +7), so a CTA
+// has its whole 32 KB tile in flight before any arithmetic.
+//   ROWS: 1x128 groups along K (the tile's columns) -> q[M][K], s[K/128][M]; each
+//         half-warp holds one row, reduced with a 16-lane shuffle.
+//   COLS: 1x128 groups along M (the tile's rows) -> qt[K][M], st[M/128][K]; the tile
+//         goes through shared memory, thread t takes column pair t%64 over rows
+//         32*(t/64) .. +31 (conflict-free 4-byte reads), the four row quarters meet
+//         in shared memory for the column absmax.
+// With both, X is read once for the two layouts wgrad and fprop/dgrad need.
+constexpr int QD_THREADS = 256;
+
+template <bool ROWS, bool COLS>
+__global__ void __launch_bounds__(QD_THREADS)
+quant_tile_kernel(const uint4 *__restrict__ x, int64_t M, int64_t K, uint2 *__restrict__ q,
+                  float *__restrict__ s, uint8_t *__restrict__ qt, float *__restrict__ st)
+{
+    __shared__ uint32_t tile[COLS ? 128 * 64 : 1];
+    __shared__ uint32_t red[4][64];
+    const int t = threadIdx.x;
+    const int64_t kb = blockIdx.x, mb = blockIdx.y;
+    const int rsub = t >> 4, sub = t & 15;
+
+    uint4 v[8];
+#pragma unroll
+    for (int p = 0; p < 8; ++p) {
+        const int64_t m = mb * 128 + p * 16 + rsub;
+        v[p] = __ldg(x + (m * K + kb * 128) / 8 + sub);
+    }
+#pragma unroll
+    for (int p = 0; p < 8; ++p) {
+        const int row = p * 16 + rsub;
+        if (ROWS) {
+            uint32_t m2 = __vmaxu2(absmax2(v[p].x, v[p].y), absmax2(v[p].z, v[p].w));
+#pragma unroll
+            for (int o = 8; o >= 1; o >>= 1)
+                m2 = __vmaxu2(m2, __shfl_xor_sync(0xffffffffu, m2, o));
+            const float amax = halves_max_to_float(m2);
+            const float sc = __fdiv_rn(amax, 448.0f);
+            uint2 codes = make_uint2(0u, 0u);
+            if (amax != 0.0f)
+                codes = quant8(v[p], GroupDiv(sc));
+            const int64_t m = mb * 128 + row;
+            q[(m * K + kb * 128) / 8 + sub] = codes;
+            if (sub == 0)
+                s[kb * M + m] = sc;
+        }
+        if (COLS)
+            *reinterpret_cast<uint4 *>(&tile[row * 64 + sub * 4]) = v[p];
+    }
+    if (COLS) {
+        __syncthreads();
+        const int cp = t & 63, rq = t >> 6;
+        uint32_t w[32];
+#pragma unroll
+        for (int i = 0; i < 32; ++i)
+            w[i] = tile[(rq * 32 + i) * 64 + cp];
+        uint32_t m2 = 0;
+#pragma unroll
+        for (int i = 0; i < 32; i += 2)
+            m2 = __vmaxu2(m2, absmax2(w[i], w[i + 1]));
+        red[rq][cp] = m2;
+        __syncthreads();
+        m2 = __vmaxu2(__vmaxu2(red[0][cp], red[1][cp]), __vmaxu2(red[2][cp], red[3][cp]));
+        const float amax_lo = __uint_as_float((m2 & 0xFFFFu) << 16);
+        const float amax_hi = __uint_as_float(m2 & 0xFFFF0000u);
+        const float s_lo = __fdiv_rn(amax_lo, 448.0f);
+        const float s_hi = __fdiv_rn(amax_hi, 448.0f);
+        uint32_t clo[8], chi[8];
+#pragma unroll
+        for (int i = 0; i < 8; ++i)
+            clo[i] = chi[i] = 0u;
+        const GroupDiv dlo(s_lo), dhi(s_hi);
+        if (dlo.fast && dhi.fast) {
+            const float2 r2 = make_float2(dlo.r, dhi.r), ns2 = make_float2(-s_lo, -s_hi);
+#pragma unroll
+            for (int i = 0; i < 32; i += 2) {
+                const float2 a = div2_fast(make_float2(bf16lo(w[i]), bf16hi(w[i])), r2, ns2);
+                const float2 b = div2_fast(make_float2(bf16lo(w[i + 1]), bf16hi(w[i + 1])), r2, ns2);
+                clo[i / 4] |= cvt_e4m3x2(a.x, b.x) << (16 * ((i / 2) & 1));
+                chi[i / 4] |= cvt_e4m3x2(a.y, b.y) << (16 * ((i / 2) & 1));
+            }
+        } else {
+#pragma unroll
+            for (int i = 0; i < 32; i += 2) {
+                clo[i / 4] |= cvt_e4m3x2(__fdiv_rn(bf16lo(w[i]), s_lo),
+                                         __fdiv_rn(bf16lo(w[i + 1]), s_lo))
+                              << (16 * ((i / 2) & 1));
+                chi[i / 4] |= cvt_e4m3x2(__fdiv_rn(bf16hi(w[i]), s_hi),
+                                         __fdiv_rn(bf16hi(w[i + 1]), s_hi))
+                              << (16 * ((i / 2) & 1));
+            }
+        }
+        if (amax_lo == 0.0f) {
+#pragma unroll
+            for (int i = 0; i < 8; ++i)
+                clo[i] = 0u;
+        }
+        if (amax_hi == 0.0f) {
+#pragma unroll
+            for (int i = 0; i < 8; ++i)
+                chi[i] = 0u;
+        }
+        const int64_t col = kb * 128 + 2 * cp;
+        const int64_t m0 = mb * 128 + rq * 32;
+        uint4 *dlo_p = reinterpret_cast<uint4 *>(qt + col * M + m0);
+        uint4 *dhi_p = reinterpret_cast<uint4 *>(qt + (col + 1) * M + m0);
+        dlo_p[0] = make_uint4(clo[0], clo[1], clo[2], clo[3]);
+        dlo_p[1] = make_uint4(clo[4], clo[5], clo[6], clo[7]);
+        dhi_p[0] = make_uint4(chi[0], chi[1], chi[2], chi[3]);
+        dhi_p[1] = make_uint4(chi[4], chi[5], chi[6], chi[7]);
+        if (rq == 0)
+            *reinterpret_cast<float2 *>(st + mb * K + col) = make_float2(s_lo, s_hi);
+    }
+}
+
 // ------------------------------------------------------------------ launchers
+
+#ifndef FP8BW_QUANT_TILE
+#define FP8BW_QUANT_TILE 1
+#endif
 
 cudaError_t launch_quant_act(const void *x, int64_t M, int64_t K, uint8_t *q, float *s,
                              cudaStream_t stream, int num_sms)
 {
+    if (FP8BW_QUANT_TILE) {
+        dim3 grid(unsigned(K / 128), unsigned(M / 128));
+        quant_tile_kernel<true, false><<<grid, QD_THREADS, 0, stream>>>(
+            static_cast<const uint4 *>(x), M, K, reinterpret_cast<uint2 *>(q), s, nullptr,
+            nullptr);
+        return cudaGetLastError();
+    }
     const int64_t npairs = M * (K / 128) / 2;
     const int64_t warps_needed = (npairs + QA_UNROLL - 1) / QA_UNROLL;
     int64_t blocks = (warps_needed + (QA_THREADS / 32) - 1) / (QA_THREADS / 32);
@@ -313,9 +442,24 @@ cudaError_t launch_quant_act(const void *x, int64_t M, int64_t K, uint8_t *q, fl
     return cudaGetLastError();
 }
 
+cudaError_t launch_quant_dual(const void *x, int64_t M, int64_t K, uint8_t *q, float *s,
+                              uint8_t *qt, float *st, cudaStream_t stream)
+{
+    dim3 grid(unsigned(K / 128), unsigned(M / 128));
+    quant_tile_kernel<true, true><<<grid, QD_THREADS, 0, stream>>>(
+        static_cast<const uint4 *>(x), M, K, reinterpret_cast<uint2 *>(q), s, qt, st);
+    return cudaGetLastError();
+}
+
 cudaError_t launch_quant_act_t(const void *x, int64_t M, int64_t K, uint8_t *qt, float *st,
                                cudaStream_t stream)
 {
+    if (FP8BW_QUANT_TILE) {
+        dim3 grid(unsigned(K / 128), unsigned(M / 128));
+        quant_tile_kernel<false, true><<<grid, QD_THREADS, 0, stream>>>(
+            static_cast<const uint4 *>(x), M, K, nullptr, nullptr, qt, st);
+        return cudaGetLastError();
+    }
     dim3 grid(unsigned(K / 64), unsigned(M / 128));
     quant_act_t_kernel<<<grid, QT_THREADS, 0, stream>>>(static_cast<const uint32_t *>(x), M, K,
                                                        qt, st);

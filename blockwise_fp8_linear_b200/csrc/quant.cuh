@@ -10,6 +10,8 @@ cudaError_t launch_quant_act(const void *x, int64_t M, int64_t K, uint8_t *q, fl
                              cudaStream_t stream, int num_sms);
 cudaError_t launch_quant_act_t(const void *x, int64_t M, int64_t K, uint8_t *qt, float *st,
                                cudaStream_t stream);
+cudaError_t launch_quant_dual(const void *x, int64_t M, int64_t K, uint8_t *q, float *s,
+                              uint8_t *qt, float *st, cudaStream_t stream);
 cudaError_t launch_quant_weight(const void *w, int64_t N, int64_t K, uint8_t *q, float *s,
                                 uint8_t *qt, cudaStream_t stream);
 

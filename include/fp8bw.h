@@ -87,6 +87,19 @@ int fp8_quant_act_t(const void *x_bf16, int64_t M, int64_t K, uint8_t *qt, float
                     void *stream);
 
 /*
+ * fp8_quant_act_dual -- both activation layouts from one read of X (section 3.2:
+ * the layer's quantized input is retained for wgrad; this produces, in one pass over
+ * the BF16 tensor, the row-wise copy fprop/dgrad consume and the token-wise copy
+ * wgrad consumes).  Outputs are bit-identical to fp8_quant_act(x, M, K, q, s) and
+ * fp8_quant_act_t(x, M, K, qt, st):
+ *   x [M][K] BF16 in
+ *   q [M][K], s [K/128][M]      1x128 groups along K
+ *   qt [K][M], st [M/128][K]    1x128 groups along M (codes transposed)
+ */
+int fp8_quant_act_dual(const void *x_bf16, int64_t M, int64_t K, uint8_t *q, float *s,
+                       uint8_t *qt, float *st, void *stream);
+
+/*
  * fp8_quant_weight -- 128x128 blocks (section 3.2: "weights use two-dimensional
  * 128x128 blocks").
  *   w  [N][K] BF16 in      q [N][K] E4M3 out      s [N/128][K/128] FP32 out

@@ -7,7 +7,8 @@ import pytest
 import torch
 
 import oracle
-from blockwise_fp8_linear_b200 import fp8_quant_act, fp8_quant_act_t, fp8_quant_weight, synth
+from blockwise_fp8_linear_b200 import (fp8_quant_act, fp8_quant_act_dual, fp8_quant_act_t,
+                                       fp8_quant_weight, synth)
 from tests._gpu import to_dev_bf16
 
 pytestmark = pytest.mark.gpu
@@ -42,6 +43,19 @@ def test_quant_act_t_parity(M, K):
     qr, sr = oracle.quant_act_t(x)
     _eq_bits(qt, qr, "codes")
     _eq_bits(st, sr, "scales")
+
+
+@pytest.mark.parametrize("M,K", ACT_SHAPES)
+def test_quant_act_dual_parity(M, K):
+    """One read, both layouts: each bit-identical to the oracle's own quantizer."""
+    x = synth.normal_bf16(M, K, 1.0, seed=synth.seed_for(4, M + K), outliers=True)
+    q, s, qt, st = fp8_quant_act_dual(to_dev_bf16(x))
+    qr, sr = oracle.quant_act(x)
+    qtr, str_ = oracle.quant_act_t(x)
+    _eq_bits(q, qr, "row codes")
+    _eq_bits(s, sr, "row scales")
+    _eq_bits(qt, qtr, "token codes")
+    _eq_bits(st, str_, "token scales")
 
 
 @pytest.mark.parametrize("N,K,want_t", [(1024, 1024, False), (384, 640, True), (4096, 2048, True),
@@ -84,6 +98,13 @@ def test_quant_edge_cases_all_layouts():
     qt, st = fp8_quant_act_t(to_dev_bf16(xt))
     qtr, str_ = oracle.quant_act_t(xt)
     _eq_bits(qt, qtr, "act_t codes"); _eq_bits(st, str_, "act_t scales")
+    for arr in (x, xt):
+        a = np.ascontiguousarray(arr)
+        q, s, qt, st = fp8_quant_act_dual(to_dev_bf16(a))
+        qr, sr = oracle.quant_act(a)
+        qtr, str_ = oracle.quant_act_t(a)
+        _eq_bits(q, qr, "dual row codes"); _eq_bits(s, sr, "dual row scales")
+        _eq_bits(qt, qtr, "dual token codes"); _eq_bits(st, str_, "dual token scales")
     for blk in (x, xt):
         w = np.ascontiguousarray(blk)
         q, s, qt = fp8_quant_weight(to_dev_bf16(w), want_t=True)
