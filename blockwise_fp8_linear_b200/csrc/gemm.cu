@@ -94,6 +94,11 @@ struct GemmCfg {
     // stores; each epilogue warp owns 32 rows x COLS columns of BF16 staging, laid
     // out as 64-column boxes of 32 rows x 128 B with the 128-byte swizzle.
     static constexpr bool TMA_STORE = (CG == 2);
+    // wgrad on the pair path promotes from the 16x256b TMEM layout (see the epilogue)
+#ifndef FP8BW_WG16
+#define FP8BW_WG16 1
+#endif
+    static constexpr bool WG16 = FP8BW_WG16 && MODE == 2 && TMA_STORE && COLS == 128;
     static constexpr int STAGE_OUT_WARP = 32 * COLS * 2;
     static constexpr int OUT_BYTES = TMA_STORE ? EPI_WARPS * STAGE_OUT_WARP : 0;
     static constexpr int RING_OFF = STAGES * STAGE_BYTES + OUT_BYTES;
@@ -367,47 +372,96 @@ fp8_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__
             const float sc = (MODE == 2) ? a_s : a_s * slot[BM + col0 / 128];
             const float2 sc2 = make_float2(sc, sc);
 
-            // TMEM -> registers in 32-column chunks; with 64 columns per thread both
-            // chunks are loaded before one wait.  The buffer goes back to the MMA as
-            // soon as the last chunk is in registers.
-            constexpr int CHUNKS = COLS / 32;
-            constexpr int GRP = (CHUNKS <= 2) ? CHUNKS : 1;
+            if constexpr (Cfg::WG16) {
+                // wgrad, 16x256b layout: thread (t0, t1) = (lane % 4, lane / 4) holds
+                // rows t1 + 8i (i < 4) of the warp's 32 and columns 64cc + 8j + 2t0 + {0,1}
+                // (cc < 2, j < 8) of its 128, so each column-scale pair read from shared
+                // memory serves four rows.
+                const int t0 = lane & 3, t1 = lane >> 2;
+                float2 sa2[4];
 #pragma unroll
-            for (int cg = 0; cg < CHUNKS; cg += GRP) {
-                uint32_t v[GRP][32];
-#pragma unroll
-                for (int g = 0; g < GRP; ++g)
-                    tmem_ld_32x32b_x32(taddr + uint32_t((cg + g) * 32), v[g]);
-                tmem_wait_ld();
-                if (cg + GRP == CHUNKS) {
-                    tc_fence_before();
-                    __syncwarp();
-                    if (lane == 0) {
-                        if (CG == 1 || rank == 0)
-                            mbar_arrive(&tempty[buf]);
-                        else  // the MMA issuer lives in the even CTA
-                            mbar_arrive_cluster(tempty_lead + uint32_t(buf) * 8u);
-                    }
+                for (int i = 0; i < 4; ++i) {
+                    const float v = slot[quarter * 32 + t1 + 8 * i];
+                    sa2[i] = make_float2(v, v);
                 }
 #pragma unroll
-                for (int g = 0; g < GRP; ++g) {
-                    const int c = cg + g;
+                for (int cc = 0; cc < 2; ++cc) {
+                    float2 sbp[8];
 #pragma unroll
-                    for (int jj = 0; jj < 16; jj += 2) {
-                        const float2 p0 = make_float2(__uint_as_float(v[g][2 * jj]),
-                                                      __uint_as_float(v[g][2 * jj + 1]));
-                        const float2 p1 = make_float2(__uint_as_float(v[g][2 * jj + 2]),
-                                                      __uint_as_float(v[g][2 * jj + 3]));
-                        float2 &a0 = acc[c * 16 + jj];
-                        float2 &a1 = acc[c * 16 + jj + 1];
-                        if (MODE == 2) {
-                            const float4 bs = *reinterpret_cast<const float4 *>(
-                                slot + BM + col0 + c * 32 + 2 * jj);
-                            a0 = __ffma2_rn(__fmul2_rn(p0, make_float2(bs.x, bs.y)), sc2, a0);
-                            a1 = __ffma2_rn(__fmul2_rn(p1, make_float2(bs.z, bs.w)), sc2, a1);
-                        } else {
-                            a0 = __ffma2_rn(p0, sc2, a0);
-                            a1 = __ffma2_rn(p1, sc2, a1);
+                    for (int j = 0; j < 8; ++j)
+                        sbp[j] = *reinterpret_cast<const float2 *>(slot + BM + col0 + 64 * cc +
+                                                                   8 * j + 2 * t0);
+#pragma unroll
+                    for (int h = 0; h < 2; ++h) {
+                        uint32_t v[32];
+                        tmem_ld_16x256b_x8(taddr + (uint32_t(16 * h) << 16) + uint32_t(64 * cc), v);
+                        tmem_wait_ld();
+                        if (cc == 1 && h == 1) {
+                            tc_fence_before();
+                            __syncwarp();
+                            if (lane == 0) {
+                                if (CG == 1 || rank == 0)
+                                    mbar_arrive(&tempty[buf]);
+                                else
+                                    mbar_arrive_cluster(tempty_lead + uint32_t(buf) * 8u);
+                            }
+                        }
+#pragma unroll
+                        for (int j = 0; j < 8; ++j) {
+#pragma unroll
+                            for (int e = 0; e < 2; ++e) {
+                                const int i = 2 * h + e;
+                                const float2 p = make_float2(__uint_as_float(v[4 * j + 2 * e]),
+                                                             __uint_as_float(v[4 * j + 2 * e + 1]));
+                                float2 &a = acc[i * 16 + cc * 8 + j];
+                                a = __ffma2_rn(__fmul2_rn(p, sbp[j]), sa2[i], a);
+                            }
+                        }
+                    }
+                }
+            } else {
+            // TMEM -> registers in 32-column chunks; with 64 columns per thread both
+                // chunks are loaded before one wait.  The buffer goes back to the MMA as
+                // soon as the last chunk is in registers.
+                constexpr int CHUNKS = COLS / 32;
+                constexpr int GRP = (CHUNKS <= 2) ? CHUNKS : 1;
+    #pragma unroll
+                for (int cg = 0; cg < CHUNKS; cg += GRP) {
+                    uint32_t v[GRP][32];
+    #pragma unroll
+                    for (int g = 0; g < GRP; ++g)
+                        tmem_ld_32x32b_x32(taddr + uint32_t((cg + g) * 32), v[g]);
+                    tmem_wait_ld();
+                    if (cg + GRP == CHUNKS) {
+                        tc_fence_before();
+                        __syncwarp();
+                        if (lane == 0) {
+                            if (CG == 1 || rank == 0)
+                                mbar_arrive(&tempty[buf]);
+                            else  // the MMA issuer lives in the even CTA
+                                mbar_arrive_cluster(tempty_lead + uint32_t(buf) * 8u);
+                        }
+                    }
+    #pragma unroll
+                    for (int g = 0; g < GRP; ++g) {
+                        const int c = cg + g;
+    #pragma unroll
+                        for (int jj = 0; jj < 16; jj += 2) {
+                            const float2 p0 = make_float2(__uint_as_float(v[g][2 * jj]),
+                                                          __uint_as_float(v[g][2 * jj + 1]));
+                            const float2 p1 = make_float2(__uint_as_float(v[g][2 * jj + 2]),
+                                                          __uint_as_float(v[g][2 * jj + 3]));
+                            float2 &a0 = acc[c * 16 + jj];
+                            float2 &a1 = acc[c * 16 + jj + 1];
+                            if (MODE == 2) {
+                                const float4 bs = *reinterpret_cast<const float4 *>(
+                                    slot + BM + col0 + c * 32 + 2 * jj);
+                                a0 = __ffma2_rn(__fmul2_rn(p0, make_float2(bs.x, bs.y)), sc2, a0);
+                                a1 = __ffma2_rn(__fmul2_rn(p1, make_float2(bs.z, bs.w)), sc2, a1);
+                            } else {
+                                a0 = __ffma2_rn(p0, sc2, a0);
+                                a1 = __ffma2_rn(p1, sc2, a1);
+                            }
                         }
                     }
                 }
@@ -422,6 +476,24 @@ fp8_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__
                     if (lane == 0)
                         bulk_wait_read0();  // the previous tile's stores have read it
                     __syncwarp();
+                    if constexpr (Cfg::WG16) {
+                        // rows t1 + 8i, columns 64cc + 8j + 2t0: one 4-byte store each,
+                        // into chunk j of box cc (conflict-free under the swizzle)
+                        const int t0 = lane & 3, t1 = lane >> 2;
+#pragma unroll
+                        for (int i = 0; i < 4; ++i)
+#pragma unroll
+                            for (int cc = 0; cc < 2; ++cc)
+#pragma unroll
+                                for (int j = 0; j < 8; ++j) {
+                                    const int row = t1 + 8 * i;
+                                    __nv_bfloat162 h =
+                                        __float22bfloat162_rn(acc[i * 16 + cc * 8 + j]);
+                                    *reinterpret_cast<uint32_t *>(
+                                        stg + cc * 4096 + row * 128 + ((j ^ (row & 7)) << 4) +
+                                        4 * t0) = *reinterpret_cast<uint32_t *>(&h);
+                                }
+                    } else {
 #pragma unroll
                     for (int c = 0; c < COLS / 8; ++c) {
                         uint4 o;
@@ -436,6 +508,7 @@ fp8_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__
                         const int box = c >> 3, chunk = c & 7;
                         *reinterpret_cast<uint4 *>(stg + box * 4096 + lane * 128 +
                                                    ((chunk ^ (lane & 7)) << 4)) = o;
+                    }
                     }
                     fence_proxy_async_smem();
                     __syncwarp();
