@@ -256,11 +256,13 @@ def barrier(world):
 
 
 def max_over_ranks(x, world):
+    """Max of a per-rank number over all ranks (the slowest rank's time)."""
     if world == 1:
         return x
     import torch
     import torch.distributed as dist
-    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dev = "cuda" if dist.get_backend() == "nccl" else "cpu"
+    t = torch.tensor([x], dtype=torch.float64, device=dev)
     dist.all_reduce(t, op=dist.ReduceOp.MAX)
     return float(t.item())
 
@@ -468,7 +470,7 @@ def run_reference(args):
 
 
 KERNEL_CASES = ("gemm_fprop", "gemm_dgrad", "gemm_wgrad", "quant_act", "quant_act_t",
-                "quant_weight")
+                "quant_dual", "quant_weight")
 
 
 def run_kernel_only(args):
@@ -511,9 +513,12 @@ def run_kernel_only(args):
             launch = lambda: fb.fp8_quant_act(X)
         elif case == "quant_act_t":
             launch = lambda: fb.fp8_quant_act_t(X)
+        elif case == "quant_dual":
+            launch = lambda: fb.fp8_quant_act_dual(X)
         else:
             launch = lambda: fb.fp8_quant_weight(X)
-        work = ("GB/s", R * C * (3 + 4 / 128) / 1e9)
+        per_elem = (4 + 8 / 128) if case == "quant_dual" else (3 + 4 / 128)
+        work = ("GB/s", R * C * per_elem / 1e9)
     torch.cuda.synchronize()
     for _ in range(args.warmup):
         launch()

@@ -20,8 +20,9 @@ import os
 __all__ = [
     "FPROP", "DGRAD", "WGRAD", "Fp8bwError", "lib", "library_path",
     "fp8_quant_act", "fp8_quant_act_t", "fp8_quant_act_dual", "fp8_quant_weight",
-    "fp8_gemm_blockwise",
+    "fp8_gemm_blockwise", "fp8_gemm_wgrad_acc32",
     "fp8bw_status_string", "fp8bw_last_device_error", "fp8bw_version",
+    "fp8bw_selftest_wait_timeout",
     "linear_fprop", "linear_dgrad", "linear_wgrad",
 ]
 
@@ -53,13 +54,16 @@ def lib():
         L.fp8_quant_act_dual.argtypes = [vp, i64, i64, vp, vp, vp, vp, vp]
         L.fp8_quant_weight.argtypes = [vp, i64, i64, vp, vp, vp, vp]
         L.fp8_gemm_blockwise.argtypes = [i32, vp, vp, vp, vp, vp, i64, i64, i64, vp]
+        L.fp8_gemm_wgrad_acc32.argtypes = [vp, vp, vp, vp, vp, i64, i64, i64, vp]
         for f in (L.fp8_quant_act, L.fp8_quant_act_t, L.fp8_quant_act_dual, L.fp8_quant_weight,
-                  L.fp8_gemm_blockwise):
+                  L.fp8_gemm_blockwise, L.fp8_gemm_wgrad_acc32):
             f.restype = i32
         L.fp8bw_status_string.argtypes = [i32]
         L.fp8bw_status_string.restype = C.c_char_p
         L.fp8bw_last_device_error.argtypes = [vp]
         L.fp8bw_last_device_error.restype = i32
+        L.fp8bw_selftest_wait_timeout.argtypes = [i64, vp]
+        L.fp8bw_selftest_wait_timeout.restype = i32
         L.fp8bw_version.argtypes = []
         L.fp8bw_version.restype = C.c_char_p
         _lib = L
@@ -99,6 +103,12 @@ def _need(t, dtype, ndim, name):
 def fp8bw_last_device_error(stream=None) -> int:
     """Synchronize the stream and return (and clear) the device error word status."""
     return int(lib().fp8bw_last_device_error(_stream(stream)))
+
+
+def fp8bw_selftest_wait_timeout(limit_us: int, stream=None) -> None:
+    """Run the bounded-wait self-test kernel (a wait that nothing satisfies)."""
+    _check(lib().fp8bw_selftest_wait_timeout(int(limit_us), _stream(stream)),
+           "fp8bw_selftest_wait_timeout")
 
 
 def fp8_quant_act(x, q=None, s=None, stream=None):
@@ -166,6 +176,20 @@ def fp8_gemm_blockwise(mode: int, a, sa, b, sb, M: int, N: int, K: int, out=None
                                     sb.data_ptr(), out.data_ptr(), M, N, K, _stream(stream)),
            "fp8_gemm_blockwise")
     return out
+
+
+def fp8_gemm_wgrad_acc32(a, sa, b, sb, M: int, N: int, K: int, dw32, stream=None):
+    """dw32[M][N] (float32, caller-owned) += the wgrad sum, kept in FP32 (no BF16
+    rounding); a, sa, b, sb as for fp8_gemm_blockwise(WGRAD, ...)."""
+    import torch
+    for t, dt, name in ((a, torch.uint8, "a"), (b, torch.uint8, "b"),
+                        (sa, torch.float32, "sa"), (sb, torch.float32, "sb"),
+                        (dw32, torch.float32, "dw32")):
+        _need(t, dt, 2, name)
+    _check(lib().fp8_gemm_wgrad_acc32(a.data_ptr(), sa.data_ptr(), b.data_ptr(), sb.data_ptr(),
+                                      dw32.data_ptr(), M, N, K, _stream(stream)),
+           "fp8_gemm_wgrad_acc32")
+    return dw32
 
 
 # -- the three GEMMs of the linear layer, composed from the entry points above ----

@@ -177,6 +177,23 @@ int fp8_gemm_blockwise(int mode, const uint8_t *a, const float *sa, const uint8_
                                         static_cast<cudaStream_t>(stream), sms));
 }
 
+int fp8_gemm_wgrad_acc32(const uint8_t *a, const float *sa, const uint8_t *b, const float *sb,
+                         float *dw32, int64_t M, int64_t N, int64_t K, void *stream)
+{
+    if (!a || !sa || !b || !sb || !dw32)
+        return FP8BW_EINVAL;
+    if (!dim_ok(M) || !dim_ok(N) || !dim_ok(K))
+        return FP8BW_ESHAPE;
+    if (!aligned16(a) || !aligned16(sa) || !aligned16(b) || !aligned16(sb) || !aligned16(dw32))
+        return FP8BW_EALIGN;
+    int st;
+    const int sms = device_sms({a, sa, b, sb, dw32}, &st);
+    if (sms < 0)
+        return st;
+    return from_cuda(fp8bw::launch_gemm_wgrad_acc32(a, sa, b, sb, dw32, M, N, K,
+                                                    static_cast<cudaStream_t>(stream), sms));
+}
+
 const char *fp8bw_status_string(int status)
 {
     switch (status) {
@@ -200,6 +217,17 @@ int fp8bw_last_device_error(void *stream)
     if (fp8bw::read_and_clear_device_error(static_cast<cudaStream_t>(stream), &v) != cudaSuccess)
         return FP8BW_ECUDA;
     return v ? FP8BW_ETIMEOUT : FP8BW_OK;
+}
+
+int fp8bw_selftest_wait_timeout(int64_t limit_us, void *stream)
+{
+    if (limit_us < 1 || limit_us > 1000000)
+        return FP8BW_EINVAL;
+    int st;
+    if (device_sms({}, &st) < 0)
+        return st;
+    return from_cuda(fp8bw::launch_selftest_wait(uint64_t(limit_us) * 1000u,
+                                                 static_cast<cudaStream_t>(stream)));
 }
 
 const char *fp8bw_version(void)

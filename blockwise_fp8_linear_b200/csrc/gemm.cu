@@ -53,12 +53,15 @@ constexpr uint64_t DRAIN_NS = 20000000ull;
 
 enum : int { ERR_PRODUCER = 1, ERR_MMA_FULL = 2, ERR_MMA_TEMPTY = 3, ERR_EPI = 4, ERR_SCALES = 5 };
 
-template <int BN_, int MODE_, int STAGES_, int CG_>
+template <int BN_, int MODE_, int STAGES_, int CG_, bool OUT32_ = false>
 struct GemmCfg {
     static constexpr int BN = BN_;      // columns of D per tile (both CTAs of a pair)
     static constexpr int MODE = MODE_;  // 0 fprop, 1 dgrad (B is MN-major), 2 wgrad
     static constexpr int STAGES = STAGES_;
     static constexpr int CG = CG_;      // CTAs per MMA (1 or 2)
+    // OUT32: instead of storing BF16, add the FP32 sum into an FP32 output (wgrad
+    // main-grad accumulation; TMA reduce-add on the pair path)
+    static constexpr bool OUT32 = OUT32_;
     static constexpr int TILE_M = BM * CG;
     static constexpr int EPI_WARPS = 8;
     static constexpr int COLS = 4 * BN / EPI_WARPS;  // columns per epilogue thread
@@ -99,6 +102,7 @@ struct GemmCfg {
 #define FP8BW_WG16 1
 #endif
     static constexpr bool WG16 = FP8BW_WG16 && MODE == 2 && TMA_STORE && COLS == 128;
+    static_assert(!OUT32 || (MODE == 2 && (WG16 || !TMA_STORE)), "FP32 output is wgrad-only");
     static constexpr int STAGE_OUT_WARP = 32 * COLS * 2;
     static constexpr int OUT_BYTES = TMA_STORE ? EPI_WARPS * STAGE_OUT_WARP : 0;
     static constexpr int RING_OFF = STAGES * STAGE_BYTES + OUT_BYTES;
@@ -129,10 +133,12 @@ template <class Cfg>
 __global__ void __launch_bounds__(Cfg::THREADS, 1)
 fp8_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                 const __grid_constant__ CUtensorMap tmD, const float *__restrict__ sa, const float *__restrict__ sb,
-                __nv_bfloat16 *__restrict__ D, int M, int N, int K)
+                void *__restrict__ Dv, int M, int N, int K)
 {
     constexpr int BN = Cfg::BN, MODE = Cfg::MODE, STAGES = Cfg::STAGES, CG = Cfg::CG;
     constexpr int COLS = Cfg::COLS, EPI_WARPS = Cfg::EPI_WARPS;
+    __nv_bfloat16 *D = static_cast<__nv_bfloat16 *>(Dv);
+    float *D32 = static_cast<float *>(Dv);
 
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>(
@@ -470,7 +476,49 @@ fp8_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__
             if (lane == 0)
                 mbar_arrive(&sempty[r]);  // this warp is done with the slot's scales
             if (++kb == KB) {
-                if (Cfg::TMA_STORE) {
+                if constexpr (Cfg::OUT32 && Cfg::TMA_STORE) {
+                    // FP32 tile -> swizzled staging (32 rows x 64 columns per pass, two
+                    // 32x32 boxes) -> bulk tensor reduce-add into the FP32 output.
+                    uint8_t *stg = sout + ew * Cfg::STAGE_OUT_WARP;
+                    const int t0 = lane & 3, t1 = lane >> 2;
+                    const int r0 = tm * Cfg::TILE_M + rank * BM + quarter * 32;
+#pragma unroll
+                    for (int cc = 0; cc < 2; ++cc) {
+                        if (lane == 0)
+                            bulk_wait_read0();
+                        __syncwarp();
+#pragma unroll
+                        for (int i = 0; i < 4; ++i)
+#pragma unroll
+                            for (int j = 0; j < 8; ++j) {
+                                const int row = t1 + 8 * i;
+                                const int chunk = 2 * (j & 3) + (t0 >> 1);
+                                *reinterpret_cast<float2 *>(stg + (j >> 2) * 4096 + row * 128 +
+                                                            ((chunk ^ (row & 7)) << 4) +
+                                                            8 * (t0 & 1)) =
+                                    acc[i * 16 + cc * 8 + j];
+                            }
+                        fence_proxy_async_smem();
+                        __syncwarp();
+                        if (lane == 0) {
+                            tma_reduce_add_2d(&tmD, stg, tn * BN + col0 + 64 * cc, r0);
+                            tma_reduce_add_2d(&tmD, stg + 4096, tn * BN + col0 + 64 * cc + 32, r0);
+                            bulk_commit();
+                        }
+                    }
+                } else if constexpr (Cfg::OUT32) {
+                    float *dst = D32 + size_t(tm * Cfg::TILE_M + row_in_tile) * size_t(N) +
+                                 size_t(tn * BN + col0);
+#pragma unroll
+                    for (int c = 0; c < COLS / 4; ++c) {
+                        float4 o = *reinterpret_cast<const float4 *>(dst + 4 * c);
+                        o.x += acc[2 * c].x;
+                        o.y += acc[2 * c].y;
+                        o.z += acc[2 * c + 1].x;
+                        o.w += acc[2 * c + 1].y;
+                        *reinterpret_cast<float4 *>(dst + 4 * c) = o;
+                    }
+                } else if (Cfg::TMA_STORE) {
                     // BF16 tile -> swizzled staging -> two bulk tensor stores per warp.
                     uint8_t *stg = sout + ew * Cfg::STAGE_OUT_WARP;
                     if (lane == 0)
@@ -628,6 +676,23 @@ static bool make_map_bf16_out(CUtensorMap *map, void *base, uint64_t rows, uint6
     return r == CUDA_SUCCESS;
 }
 
+// FP32 [rows][cols] output map for TMA reduce-add: box 32 columns (128 B) x 32 rows,
+// 128-byte swizzle.
+static bool make_map_f32_out(CUtensorMap *map, void *base, uint64_t rows, uint64_t cols)
+{
+    EncodeTiledFn enc = get_encode_fn();
+    if (!enc)
+        return false;
+    cuuint64_t gdim[2] = {cols, rows};
+    cuuint64_t gstride[1] = {cols * 4};
+    cuuint32_t box[2] = {32, 32};
+    cuuint32_t estride[2] = {1, 1};
+    CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, base, gdim, gstride, box, estride,
+                     CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                     CU_TENSOR_MAP_L2_PROMOTION_NONE, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS;
+}
+
 template <class Cfg>
 static cudaError_t run(const uint8_t *a, const float *sa, const uint8_t *b, const float *sb,
                        void *d, int64_t M, int64_t N, int64_t K, cudaStream_t stream, int num_sms)
@@ -657,10 +722,12 @@ static cudaError_t run(const uint8_t *a, const float *sa, const uint8_t *b, cons
         return cudaErrorInvalidValue;
     CUtensorMap td;
     std::memset(&td, 0, sizeof td);
-    if (Cfg::TMA_STORE && !make_map_bf16_out(&td, d, uint64_t(M), uint64_t(N)))
+    if (Cfg::TMA_STORE && !Cfg::OUT32 && !make_map_bf16_out(&td, d, uint64_t(M), uint64_t(N)))
+        return cudaErrorInvalidValue;
+    if (Cfg::TMA_STORE && Cfg::OUT32 && !make_map_f32_out(&td, d, uint64_t(M), uint64_t(N)))
         return cudaErrorInvalidValue;
     const int64_t tiles = (M / Cfg::TILE_M) * (N / Cfg::BN);
-    __nv_bfloat16 *dp = static_cast<__nv_bfloat16 *>(d);
+    void *dp = d;
     if (Cfg::CG == 1) {
         const int grid = int(tiles < num_sms ? tiles : num_sms);
         kern<<<grid, Cfg::THREADS, Cfg::SMEM, stream>>>(ta, tb, td, sa, sb, dp, int(M), int(N),
@@ -726,6 +793,46 @@ cudaError_t launch_gemm(int mode, const uint8_t *a, const float *sa, const uint8
         return wide ? run<GemmCfg<256, 2, 4, 1>>(a, sa, b, sb, d, M, N, K, stream, num_sms)
                     : run<GemmCfg<128, 2, 6, 1>>(a, sa, b, sb, d, M, N, K, stream, num_sms);
     }
+}
+
+cudaError_t launch_gemm_wgrad_acc32(const uint8_t *a, const float *sa, const uint8_t *b,
+                                    const float *sb, float *d32, int64_t M, int64_t N, int64_t K,
+                                    cudaStream_t stream, int num_sms)
+{
+    const bool wide = (N % 256) == 0;
+    const bool pair = FP8BW_PAIR && FP8BW_WG16 && wide && (M % 256) == 0 &&
+                      (M / 256) * (N / 256) >= 16;
+    if (pair)
+        return run<GemmCfg<256, 2, 4, 2, true>>(a, sa, b, sb, d32, M, N, K, stream, num_sms);
+    return wide ? run<GemmCfg<256, 2, 4, 1, true>>(a, sa, b, sb, d32, M, N, K, stream, num_sms)
+                : run<GemmCfg<128, 2, 6, 1, true>>(a, sa, b, sb, d32, M, N, K, stream, num_sms);
+}
+
+// Self-test of the bounded-wait path: one warp waits, with the same bounded wait the
+// GEMM uses, on a shared-memory barrier that nothing ever arrives on.  The wait runs
+// out after limit_ns, records ERR_SELFTEST in the device error word and the kernel
+// returns normally; no fault, trap or unbounded wait is involved.
+enum : int { ERR_SELFTEST = 7 };
+
+__global__ void __launch_bounds__(32) selftest_wait_kernel(uint64_t limit_ns)
+{
+    __shared__ uint64_t bar;
+    __shared__ int abort_flag;
+    if (threadIdx.x == 0) {
+        mbar_init(&bar, 1);
+        abort_flag = 0;
+        fence_mbarrier_init();
+    }
+    __syncwarp();
+    if (threadIdx.x == 0)
+        mbar_wait_bounded(&bar, 0u, &abort_flag, &g_device_error, ERR_SELFTEST, limit_ns);
+    __syncwarp();
+}
+
+cudaError_t launch_selftest_wait(uint64_t limit_ns, cudaStream_t stream)
+{
+    selftest_wait_kernel<<<1, 32, 0, stream>>>(limit_ns);
+    return cudaGetLastError();
 }
 
 cudaError_t read_and_clear_device_error(cudaStream_t stream, int *value)

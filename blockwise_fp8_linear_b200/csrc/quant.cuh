@@ -21,6 +21,14 @@ cudaError_t launch_gemm(int mode, const uint8_t *a, const float *sa, const uint8
                         const float *sb, void *d, int64_t M, int64_t N, int64_t K,
                         cudaStream_t stream, int num_sms);
 
+// wgrad with FP32 main-grad accumulation: d32[M][N] += sum (no BF16 rounding).
+cudaError_t launch_gemm_wgrad_acc32(const uint8_t *a, const float *sa, const uint8_t *b,
+                                    const float *sb, float *d32, int64_t M, int64_t N, int64_t K,
+                                    cudaStream_t stream, int num_sms);
+
+// Bounded-wait self-test (records a timeout in the error word, no fault).
+cudaError_t launch_selftest_wait(uint64_t limit_ns, cudaStream_t stream);
+
 // Per-device error word written by bounded in-kernel waits.
 cudaError_t read_and_clear_device_error(cudaStream_t stream, int *value);
 

@@ -133,6 +133,19 @@ int fp8_gemm_blockwise(int mode, const uint8_t *a, const float *sa, const uint8_
                        const float *sb, void *d_bf16, int64_t M, int64_t N, int64_t K,
                        void *stream);
 
+/*
+ * fp8_gemm_wgrad_acc32 -- wgrad with FP32 gradient accumulation (the reading notes on
+ * the same paper, section 2.3: gradient accumulation stays in FP32).  Same operands
+ * and promotion as fp8_gemm_blockwise(FP8BW_WGRAD, ...), but the FP32 running sum is
+ * added into dw32 instead of being rounded to BF16:
+ *   dw32 [M][N] FP32, read and written: dw32 += sum over the token blocks
+ * (M = out_features, N = in_features, K = tokens).  Calls that overlap on the GPU and
+ * target the same dw32 may interleave their additions (the sum is the same up to
+ * FP32 rounding order).
+ */
+int fp8_gemm_wgrad_acc32(const uint8_t *a, const float *sa, const uint8_t *b, const float *sb,
+                         float *dw32, int64_t M, int64_t N, int64_t K, void *stream);
+
 /* Human-readable name of a status code (static string). */
 const char *fp8bw_status_string(int status);
 
@@ -140,6 +153,14 @@ const char *fp8bw_status_string(int status);
  * FP8BW_OK, or FP8BW_ETIMEOUT if a bounded in-kernel wait ran out since the last
  * call (the GEMM whose wait ran out returned early and its output is undefined). */
 int fp8bw_last_device_error(void *stream);
+
+/* Self-test of the failure-detection path (no counterpart in the paper; it checks
+ * this library's own bounded waits).  Launches one warp on `stream` that waits, with
+ * the GEMM's bounded wait, on a barrier nothing arrives on; after limit_us
+ * microseconds (1 .. 1e6, else FP8BW_EINVAL) the wait gives up, records a timeout in
+ * the device error word and the kernel returns.  fp8bw_last_device_error() then
+ * reports FP8BW_ETIMEOUT once; the device stays usable. */
+int fp8bw_selftest_wait_timeout(int64_t limit_us, void *stream);
 
 /* Library version, e.g. "fp8bw 0.1 sm_100a". */
 const char *fp8bw_version(void);

@@ -61,6 +61,10 @@ def test_argument_errors_before_any_launch(L):
     assert L.fp8_gemm_blockwise(0, p, p, p, p, nul, 128, 128, 128, s) == 1
     assert L.fp8_gemm_blockwise(0, p, p, p, p, p, 128, 256, 200, s) == 3
     assert L.fp8_gemm_blockwise(1, p, odd, p, p, p, 128, 256, 256, s) == 2
+    assert L.fp8_quant_act_dual(p, 128, 128, p, p, nul, p, s) == 1
+    assert L.fp8_quant_act_dual(p, 128, 100, p, p, p, p, s) == 3
+    assert L.fp8_gemm_wgrad_acc32(p, p, p, p, nul, 128, 128, 128, s) == 1
+    assert L.fp8_gemm_wgrad_acc32(p, p, p, p, odd, 128, 128, 128, s) == 2
 
 
 def test_no_gpu_reports_cuda_error_not_crash(L):

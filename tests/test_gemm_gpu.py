@@ -8,8 +8,9 @@ import pytest
 import torch
 
 import oracle
-from blockwise_fp8_linear_b200 import (DGRAD, FPROP, WGRAD, fp8_gemm_blockwise, fp8_quant_act,
-                                       fp8_quant_act_t, fp8_quant_weight, synth)
+from blockwise_fp8_linear_b200 import (DGRAD, FPROP, WGRAD, fp8_gemm_blockwise,
+                                       fp8_gemm_wgrad_acc32, fp8_quant_act, fp8_quant_act_t,
+                                       fp8_quant_weight, synth)
 from tests._gpu import bf16_dev_to_f64, check_gemm, to_dev_bf16
 
 pytestmark = pytest.mark.gpu
@@ -149,3 +150,35 @@ def test_gemm_deterministic():
     y1 = fp8_gemm_blockwise(FPROP, qx, sx, qw, sw, 1024, 2048, 2048)
     y2 = fp8_gemm_blockwise(FPROP, qx, sx, qw, sw, 1024, 2048, 2048)
     assert torch.equal(y1.view(torch.int16), y2.view(torch.int16))
+
+
+@pytest.mark.parametrize("T,Din,Dout", [
+    (256, 384, 640),      # single-CTA path, N not a multiple of 256
+    (1024, 768, 512),     # single-CTA path, 128x256 tiles
+    (8192, 2048, 4096),   # CTA-pair path (the QKV weight gradient), rows sampled
+])
+def test_wgrad_fp32_accumulation(T, Din, Dout):
+    """dW32 += wgrad sum in FP32 (gradient accumulation in FP32): starting from a
+    seeded FP32 buffer, one call adds the oracle's sum, a second call adds it again."""
+    X, W, dY = _layer(T, Din, Dout, seed=T + Din + Dout + 31)
+    a_d, sa_d = fp8_quant_act_t(to_dev_bf16(dY))
+    b_d, sb_d = fp8_quant_act_t(to_dev_bf16(X))
+    a, sa = oracle.quant_act_t(dY)
+    b, sb = oracle.quant_act_t(X)
+    for g, r in ((a_d, a), (sa_d, sa), (b_d, b), (sb_d, sb)):
+        _same(g, r)
+    M, N, K = Dout, Din, T
+    rows = _rows(M, 24) if M * N > 4 * 1024 * 1024 else None
+    rng = np.random.default_rng(7)
+    prev = (rng.standard_normal((M, N)) * 1e-3).astype(np.float32)
+    dw = torch.from_numpy(prev.copy()).cuda()
+    fp8_gemm_wgrad_acc32(a_d, sa_d, b_d, sb_d, M, N, K, dw)
+    y1 = dw.cpu().numpy().astype(np.float64)
+    fp8_gemm_wgrad_acc32(a_d, sa_d, b_d, sb_d, M, N, K, dw)
+    y2 = dw.cpu().numpy().astype(np.float64)
+    y_ref, asum = oracle.gemm(WGRAD, a, sa, b, sb, M, N, K, rows=rows)
+    p64 = prev.astype(np.float64)
+    if rows is not None:
+        y1, y2, p64 = y1[rows], y2[rows], p64[rows]
+    check_gemm(y1, p64 + y_ref, asum + np.abs(p64), "acc32 once")
+    check_gemm(y2, p64 + 2 * y_ref, 2 * asum + np.abs(p64), "acc32 twice")
