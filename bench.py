@@ -7,8 +7,15 @@ QKV (2048 -> 4096), O (2048 -> 2048), gate/up (2048 -> 12288), down (6144 -> 204
 For each linear: fp8_quant_act_dual(X) (row-wise and token-wise copies from one read),
 fp8_quant_weight(W), fprop; fp8_quant_act_dual(dY), dgrad; wgrad -- 24 kernel
 launches, 2.47 TFLOP of GEMM work (--separate-quant: the four single-layout passes,
-32 launches).  The metric is TFLOP/s of the whole step (2MNK summed over the
-12 GEMMs, divided by the time of all quantizers and GEMMs).
+32 launches).  The wgrad of each linear runs on a second stream, concurrently with
+its dgrad (both need only the quantized dY and the retained quantized X / weight), so
+that the SMs one GEMM leaves idle in its last round of tiles take the other's
+(--no-overlap: one stream).  The metric is TFLOP/s of the whole step (2MNK summed over
+the 12 GEMMs, divided by the time of all quantizers and GEMMs); the kernel roofline
+comes from a separate one-stream pass with every GEMM bracketed by events.
+
+--sweep: the micro-batch knee sweep of a 28-layer step (M = 4096 ... 32768 tokens,
+one stream), one JSON line per M and one naming the knee.
 
 Inputs are seeded synthetic BF16 tensors (X ~ N(0,1) with 1% outlier channels x20,
 W ~ N(0,0.02), dY ~ N(0,1e-3)); 637 MB per step, larger than the 126 MB L2, so no
@@ -44,8 +51,10 @@ STEP_FLOPS = sum(3 * 2 * TOKENS * din * dout for _, din, dout in LINEARS)
 FP8_OVER_BF16 = 4.5 / 2.25  # nominal dense FP8 : BF16 tensor throughput on B200
 
 
-def config_dict(n):
+def config_dict(n, overlap=True):
     return {
+        "schedule": ("each linear's wgrad on a second stream, concurrent with its dgrad"
+                     if overlap else "one stream"),
         "workload": WORKLOAD,
         "tokens": TOKENS,
         "linears": {name: [din, dout] for name, din, dout in LINEARS},
@@ -190,26 +199,32 @@ class LayerWork:
         self.h2d_bytes = sum(d[k].numel() * 2 for d in self.lin for k in ("X", "W", "dY"))
         self.d2h_bytes = sum(d[k].numel() * 2 for d in self.lin for k in ("Y", "dX", "dW"))
 
-    def step(self, gemm_events=None):
+    def step(self, gemm_events=None, side=None):
         """Enqueue one step on the current stream.  gemm_events: optional list that
-        receives (start, end, flops) CUDA-event triples around each GEMM."""
+        receives (start, end, flops) CUDA-event triples around each GEMM.  side: an
+        optional second stream; each linear's wgrad then runs there, after the dY
+        quantizer and concurrently with the dgrad (the two are independent given
+        dY), and the current stream waits for it at the end of the step."""
         fb, torch = self.fb, self.torch
         L = fb.lib()
-        st = fb._stream(None)
+        main = torch.cuda.current_stream()
         T = TOKENS
 
-        def gemm(mode, a, sa, b, sb, out, M, N, K):
+        def gemm(mode, a, sa, b, sb, out, M, N, K, stream=None):
+            s = stream if stream is not None else main
             if gemm_events is not None:
                 e0 = torch.cuda.Event(enable_timing=True)
                 e1 = torch.cuda.Event(enable_timing=True)
-                e0.record()
+                e0.record(s)
             rc = L.fp8_gemm_blockwise(mode, a.data_ptr(), sa.data_ptr(), b.data_ptr(),
-                                      sb.data_ptr(), out.data_ptr(), M, N, K, st)
+                                      sb.data_ptr(), out.data_ptr(), M, N, K, s.cuda_stream)
             if rc:
                 raise fb.Fp8bwError(rc, "fp8_gemm_blockwise")
             if gemm_events is not None:
-                e1.record()
+                e1.record(s)
                 gemm_events.append((e0, e1, 2 * M * N * K))
+
+        st = main.cuda_stream
 
         def chk(rc, what):
             if rc:
@@ -230,11 +245,19 @@ class LayerWork:
             else:
                 chk(L.fp8_quant_act_dual(d["dY"].data_ptr(), T, dout, d["qdy"].data_ptr(), d["sdy"].data_ptr(),
                                          d["qdyt"].data_ptr(), d["sdyt"].data_ptr(), st), "qd")
-            gemm(fb.DGRAD, d["qdy"], d["sdy"], d["qw"], d["sw"], d["dX"], T, din, dout)
             if self.separate:
                 chk(L.fp8_quant_act_t(d["dY"].data_ptr(), T, dout, d["qdyt"].data_ptr(), d["sdyt"].data_ptr(), st), "qt")
                 chk(L.fp8_quant_act_t(d["X"].data_ptr(), T, din, d["qxt"].data_ptr(), d["sxt"].data_ptr(), st), "qt")
-            gemm(fb.WGRAD, d["qdyt"], d["sdyt"], d["qxt"], d["sxt"], d["dW"], dout, din, T)
+            if side is not None:
+                ready = torch.cuda.Event()
+                ready.record(main)
+                side.wait_event(ready)
+            gemm(fb.DGRAD, d["qdy"], d["sdy"], d["qw"], d["sw"], d["dX"], T, din, dout)
+            gemm(fb.WGRAD, d["qdyt"], d["sdyt"], d["qxt"], d["sxt"], d["dW"], dout, din, T, stream=side)
+        if side is not None:
+            done = torch.cuda.Event()
+            done.record(side)
+            main.wait_event(done)
 
 
 def make_inputs(rank=0):
@@ -283,16 +306,32 @@ def run_ours(args):
 
     host = make_inputs(rank)
     work = LayerWork(dev, host, separate=args.separate_quant)
+    side = None if args.no_overlap else torch.cuda.Stream(device=dev)
 
     # warm-up
     for _ in range(args.warmup):
-        work.step()
+        work.step(side=side)
     torch.cuda.synchronize()
     if fb.fp8bw_last_device_error() != 0:
         raise RuntimeError("a bounded in-kernel wait ran out during warm-up")
 
-    # timed region: K steps, device time by CUDA events, GEMM launches bracketed
+    # kernel roofline: the same K steps on one stream, every GEMM launch bracketed by
+    # events, so that each launch's time is its own (no overlap with another kernel)
     gemm_events = []
+    barrier(world)
+    torch.cuda.synchronize()
+    r0 = torch.cuda.Event(enable_timing=True)
+    r1 = torch.cuda.Event(enable_timing=True)
+    r0.record()
+    for _ in range(args.steps):
+        work.step(gemm_events)
+    r1.record()
+    torch.cuda.synchronize()
+    serial_ms = r0.elapsed_time(r1)
+    gemm_ms = sum(e0.elapsed_time(e1) for e0, e1, _ in gemm_events)
+    gemm_flops = sum(f for _, _, f in gemm_events)
+
+    # timed region: K steps, device time by CUDA events on the launching stream
     with ClockSampler(dev.index) as clocks:
         barrier(world)
         torch.cuda.synchronize()
@@ -300,7 +339,7 @@ def run_ours(args):
         t1 = torch.cuda.Event(enable_timing=True)
         t0.record()
         for _ in range(args.steps):
-            work.step(gemm_events)
+            work.step(side=side)
         t1.record()
         torch.cuda.synchronize()
         barrier(world)
@@ -308,8 +347,6 @@ def run_ours(args):
     elapsed_ms = max_over_ranks(local_ms, world)
     if fb.fp8bw_last_device_error() != 0:
         raise RuntimeError("a bounded in-kernel wait ran out in the timed region")
-    gemm_ms = sum(e0.elapsed_time(e1) for e0, e1, _ in gemm_events)
-    gemm_flops = sum(f for _, _, f in gemm_events)
     clock_info = clocks.summary()
 
     ms_per_step = elapsed_ms / args.steps
@@ -331,7 +368,7 @@ def run_ours(args):
                 d["X"].view(torch.int16).copy_(X, non_blocking=True)
                 d["W"].view(torch.int16).copy_(W, non_blocking=True)
                 d["dY"].view(torch.int16).copy_(dY, non_blocking=True)
-            work.step()
+            work.step(side=side)
             for d, (Y, dX, dW) in zip(work.lin, pin_out):
                 Y.copy_(d["Y"].view(torch.int16), non_blocking=True)
                 dX.copy_(d["dX"].view(torch.int16), non_blocking=True)
@@ -364,7 +401,8 @@ def run_ours(args):
         "peak_source": f"{peak_src} cuBLAS bf16 burst x {FP8_OVER_BF16:g} (nominal FP8:BF16)",
         "traffic": recorded_traffic(),
         "traffic_unit": "bytes per GEMM launch (mean over the step's 12 GEMMs, ncu dram read+write)",
-        "gemm_share_of_step": round(gemm_ms / local_ms, 4),
+        "gemm_share_of_step": round(gemm_ms / serial_ms, 4),
+        "measured_on": "a separate pass of the same steps on one stream (no kernel overlap)",
     }
 
     cpu = None
@@ -377,7 +415,8 @@ def run_ours(args):
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_per_step, 4),
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
             "dtype": "e4m3", "data": "synthetic (seeded splitmix64/Box-Muller BF16)",
-            "config": config_dict(world), "roofline": roofline, "cpu_baseline": cpu,
+            "config": config_dict(world, overlap=side is not None), "roofline": roofline,
+            "cpu_baseline": cpu,
             "e2e": e2e, "gpu_launches": work.launches_per_step * args.steps,
             "clocks": clock_info,
             "pct_of_fp8_peak": round(100 * value / world / fp8_peak, 2),
@@ -535,6 +574,119 @@ def run_kernel_only(args):
                       work[0]: round(work[1] / (ms * 1e-3), 2)}), flush=True)
 
 
+# ------------------------------------------------- micro-batch knee sweep
+
+SWEEP_TOKENS = (4096, 8192, 16384, 32768)   # micro-batch 1, 2, 4, 8 x sequence 4096
+SWEEP_LAYERS = 28
+
+
+def run_sweep(args):
+    """Knee sweep of one 28-layer step's linear work: per layer the four linears of the
+    block in fprop + dgrad + wgrad with all quantizers (24 launches), each layer with its
+    own weights, at M = 4096 ... 32768 tokens.  Prints one JSON line per M and a
+    summary line naming the knee: the smallest M whose doubling gains < 5% of T_lin.
+    Inputs come from torch's seeded device generator (X ~ N(0,1) with 1% outlier
+    channels x20, W ~ N(0,0.02), dY ~ N(0,1e-3)); activations are shared by the
+    layers, weights are distinct per layer (2.8 GB of BF16)."""
+    import torch
+    import blockwise_fp8_linear_b200 as fb
+    from blockwise_fp8_linear_b200 import build as fbuild
+    fbuild.build()
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    L = fb.lib()
+    g = torch.Generator(device=dev).manual_seed(4)
+
+    def randn(r, c, std, outliers=False):
+        x = torch.randn(r, c, device=dev, generator=g) * std
+        if outliers:
+            cols = torch.randperm(c, device=dev, generator=g)[: c // 100]
+            x[:, cols] *= 20.0
+        return x.to(torch.bfloat16)
+
+    weights = [[randn(dout, din, 0.02) for _, din, dout in LINEARS] for _ in range(SWEEP_LAYERS)]
+    qw = [torch.empty(dout, din, dtype=torch.uint8, device=dev) for _, din, dout in LINEARS]
+    sw = [torch.empty(dout // 128, din // 128, dtype=torch.float32, device=dev) for _, din, dout in LINEARS]
+    results = []
+    for T in SWEEP_TOKENS:
+        bufs = []
+        for _, din, dout in LINEARS:
+            u8 = lambda r, c: torch.empty(r, c, dtype=torch.uint8, device=dev)
+            f32 = lambda r, c: torch.empty(r, c, dtype=torch.float32, device=dev)
+            bufs.append({
+                "X": randn(T, din, 1.0, outliers=True), "dY": randn(T, dout, 1e-3),
+                "qx": u8(T, din), "sx": f32(din // 128, T), "qxt": u8(din, T), "sxt": f32(T // 128, din),
+                "qdy": u8(T, dout), "sdy": f32(dout // 128, T), "qdyt": u8(dout, T), "sdyt": f32(T // 128, dout),
+                "Y": torch.empty(T, dout, dtype=torch.bfloat16, device=dev),
+                "dX": torch.empty(T, din, dtype=torch.bfloat16, device=dev),
+                "dW": torch.empty(dout, din, dtype=torch.bfloat16, device=dev)})
+        st = fb._stream(None)
+
+        def chk(rc, what):
+            if rc:
+                raise fb.Fp8bwError(rc, what)
+
+        def step(gemm_events=None):
+            for layer in range(SWEEP_LAYERS):
+                for i, (_, din, dout) in enumerate(LINEARS):
+                    b, W = bufs[i], weights[layer][i]
+                    p = lambda k: b[k].data_ptr()
+                    chk(L.fp8_quant_act_dual(p("X"), T, din, p("qx"), p("sx"), p("qxt"), p("sxt"), st), "qd")
+                    chk(L.fp8_quant_weight(W.data_ptr(), dout, din, qw[i].data_ptr(), sw[i].data_ptr(), None, st), "qw")
+                    chk(L.fp8_quant_act_dual(p("dY"), T, dout, p("qdy"), p("sdy"), p("qdyt"), p("sdyt"), st), "qd")
+                    for mode, a, sa, bb, sb, out, M, N, K in (
+                            (fb.FPROP, p("qx"), p("sx"), qw[i].data_ptr(), sw[i].data_ptr(), p("Y"), T, dout, din),
+                            (fb.DGRAD, p("qdy"), p("sdy"), qw[i].data_ptr(), sw[i].data_ptr(), p("dX"), T, din, dout),
+                            (fb.WGRAD, p("qdyt"), p("sdyt"), p("qxt"), p("sxt"), p("dW"), dout, din, T)):
+                        if gemm_events is not None:
+                            e0 = torch.cuda.Event(enable_timing=True)
+                            e0.record()
+                        chk(L.fp8_gemm_blockwise(mode, a, sa, bb, sb, out, M, N, K, st), "gemm")
+                        if gemm_events is not None:
+                            e1 = torch.cuda.Event(enable_timing=True)
+                            e1.record()
+                            gemm_events.append((e0, e1))
+
+        for _ in range(max(3, args.warmup)):
+            step()
+        torch.cuda.synchronize()
+        if fb.fp8bw_last_device_error() != 0:
+            raise RuntimeError("a bounded in-kernel wait ran out during the sweep warm-up")
+        ev = []
+        with ClockSampler(dev.index) as clocks:
+            t0 = torch.cuda.Event(enable_timing=True)
+            t1 = torch.cuda.Event(enable_timing=True)
+            t0.record()
+            for _ in range(args.sweep_steps):
+                step(ev)
+            t1.record()
+            torch.cuda.synchronize()
+        if fb.fp8bw_last_device_error() != 0:
+            raise RuntimeError("a bounded in-kernel wait ran out in the sweep")
+        ms = t0.elapsed_time(t1) / args.sweep_steps
+        gemm_ms = sum(a.elapsed_time(b) for a, b in ev) / args.sweep_steps
+        flops = SWEEP_LAYERS * sum(3 * 2 * T * din * dout for _, din, dout in LINEARS)
+        line = {"sweep": "micro-batch knee, 28-layer step linear work", "tokens": T,
+                "layers": SWEEP_LAYERS, "value": round(flops / (ms * 1e-3) / 1e12, 2),
+                "unit": UNIT, "ms_per_step": round(ms, 3), "step_tflop": round(flops / 1e12, 3),
+                "gemm_tflops": round(flops / (gemm_ms * 1e-3) / 1e12, 2),
+                "gemm_share_of_step": round(gemm_ms / ms, 4), "steps": args.sweep_steps,
+                "launches_per_step": SWEEP_LAYERS * 24, "clocks": clocks.summary(),
+                "data": "synthetic (torch seeded device generator)"}
+        results.append(line)
+        print(json.dumps(line), flush=True)
+        del bufs
+        torch.cuda.empty_cache()
+    knee = None
+    for a, b in zip(results, results[1:]):
+        if b["value"] < 1.05 * a["value"]:
+            knee = a["tokens"]
+            break
+    print(json.dumps({"sweep": "knee", "knee_tokens": knee,
+                      "rule": "smallest M whose doubling gains < 5% of T_lin",
+                      "values": {r["tokens"]: r["value"] for r in results}}), flush=True)
+
+
 def main():
     ap = argparse.ArgumentParser(description=__doc__.split("\n\n")[0])
     ap.add_argument("--gpus", type=int, default=1)
@@ -547,9 +699,17 @@ def main():
     ap.add_argument("--separate-quant", action="store_true",
                     help="quantize X and dY with separate row-wise and token-wise passes "
                          "instead of the fused dual-output quantizer")
+    ap.add_argument("--no-overlap", action="store_true",
+                    help="run every kernel on one stream (no dgrad/wgrad overlap)")
     ap.add_argument("--kernel-only", choices=KERNEL_CASES, default=None,
                     help="launch one kernel repeatedly (for profilers); no JSON metric line")
+    ap.add_argument("--sweep", action="store_true",
+                    help="micro-batch knee sweep (28 layers, M = 4096..32768); one JSON line per M")
+    ap.add_argument("--sweep-steps", type=int, default=3)
     args = ap.parse_args()
+    if args.sweep:
+        run_sweep(args)
+        return
     if args.kernel_only:
         run_kernel_only(args)
         return

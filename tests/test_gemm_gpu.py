@@ -127,6 +127,23 @@ def test_gemm_full_size_sampled(name, mode):
     check_gemm(y, y_ref, asum, f"{name} mode {mode}")
 
 
+# The micro-batch sweep of a 28-layer step runs the same four linears at M = 4096, 16384
+# and 32768 tokens (micro-batch 1, 4, 8 x sequence 4096): every linear at the smallest,
+# one linear at each of the larger sizes (the wgrad reduction grows to 32768 tokens).
+SWEEP = [(4096, name) for name in FULL] + [(16384, "qkv"), (32768, "down")]
+
+
+@pytest.mark.parametrize("T,name", SWEEP)
+@pytest.mark.parametrize("mode", [FPROP, DGRAD, WGRAD])
+def test_gemm_sweep_sizes_sampled(T, name, mode):
+    _, Din, Dout = FULL[name]
+    X, W, dY = _layer(T, Din, Dout, seed=T // 128 + 7 * mode + len(name))
+    M = {FPROP: T, DGRAD: T, WGRAD: Dout}[mode]
+    rows = _rows(M, 16)
+    y, y_ref, asum = _run_mode(mode, X, W, dY, rows=rows)
+    check_gemm(y, y_ref, asum, f"{name} mode {mode} M={T}")
+
+
 @pytest.mark.parametrize("mode", [FPROP, DGRAD, WGRAD])
 def test_gemm_zero_and_degenerate_inputs(mode):
     """All-zero activations give an exactly zero output; a single nonzero group
@@ -182,3 +199,4 @@ def test_wgrad_fp32_accumulation(T, Din, Dout):
         y1, y2, p64 = y1[rows], y2[rows], p64[rows]
     check_gemm(y1, p64 + y_ref, asum + np.abs(p64), "acc32 once")
     check_gemm(y2, p64 + 2 * y_ref, 2 * asum + np.abs(p64), "acc32 twice")
+
