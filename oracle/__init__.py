@@ -47,6 +47,18 @@ def _load():
                                   C.c_void_p, C.c_int64, C.c_void_p, C.c_void_p, C.c_int]
         lib.fp8o_max_threads.restype = C.c_int
         lib.fp8o_max_threads.argtypes = []
+        lib.fp8o_e8m0_exponent.restype = C.c_int
+        lib.fp8o_e8m0_exponent.argtypes = [C.c_float]
+        lib.fp8o_quantize_group_e8m0.restype = C.c_uint8
+        lib.fp8o_quantize_group_e8m0.argtypes = [C.c_void_p, C.c_int64, C.c_int64,
+                                                 C.c_void_p, C.c_int64]
+        for name in ("fp8o_quant_act_e8m0", "fp8o_quant_act_t_e8m0"):
+            f = getattr(lib, name)
+            f.restype = C.c_int
+            f.argtypes = [C.c_void_p, C.c_int64, C.c_int64, C.c_void_p, C.c_void_p]
+        lib.fp8o_quant_weight_e8m0.restype = C.c_int
+        lib.fp8o_quant_weight_e8m0.argtypes = [C.c_void_p, C.c_int64, C.c_int64, C.c_void_p,
+                                               C.c_void_p, C.c_void_p]
         _lib = lib
     return _lib
 
@@ -127,6 +139,63 @@ def quant_weight(w_bf16: np.ndarray, want_t: bool = False):
                                    _ptr(qt) if want_t else None)
     if rc:
         raise ValueError(f"oracle quant_weight: bad sizes {N}x{K}")
+    return q, s, qt
+
+
+# ---- power-of-two (E8M0) scales: the MXFP8 form of section 3.2 ----
+
+def e8m0_exponent(amax: float) -> int:
+    """Exponent e of the group scale 2^e: the smallest e with amax <= 448 * 2^e,
+    clamped to [-127, 127]; -127 for amax = 0."""
+    return int(_load().fp8o_e8m0_exponent(float(amax)))
+
+
+def e8m0_to_float(codes) -> np.ndarray:
+    """E8M0 codes (uint8, e + 127) -> the float32 scales 2^e (all exact)."""
+    c = np.asarray(codes, dtype=np.int64)
+    return np.ldexp(np.float32(1.0), (c - 127).astype(np.int32)).astype(np.float32)
+
+
+def quantize_group_e8m0(x_bf16: np.ndarray):
+    """One group of BF16 values -> (codes uint8, E8M0 scale code uint8)."""
+    x = _u16(x_bf16).ravel()
+    q = np.empty(x.size, dtype=np.uint8)
+    c = _load().fp8o_quantize_group_e8m0(_ptr(x), 1, x.size, _ptr(q), 1)
+    return q, np.uint8(c)
+
+
+def quant_act_e8m0(x_bf16: np.ndarray):
+    """X[M][K] -> (Q[M][K] uint8, S[K/128][M] uint8 E8M0 codes)."""
+    x = _u16(x_bf16)
+    M, K = x.shape
+    q = np.empty((M, K), dtype=np.uint8)
+    s = np.empty((K // 128, M), dtype=np.uint8)
+    if _load().fp8o_quant_act_e8m0(_ptr(x), M, K, _ptr(q), _ptr(s)):
+        raise ValueError(f"oracle quant_act_e8m0: bad sizes {M}x{K}")
+    return q, s
+
+
+def quant_act_t_e8m0(x_bf16: np.ndarray):
+    """X[M][K] -> (Q^T[K][M] uint8, S^T[M/128][K] uint8 E8M0 codes)."""
+    x = _u16(x_bf16)
+    M, K = x.shape
+    qt = np.empty((K, M), dtype=np.uint8)
+    st = np.empty((M // 128, K), dtype=np.uint8)
+    if _load().fp8o_quant_act_t_e8m0(_ptr(x), M, K, _ptr(qt), _ptr(st)):
+        raise ValueError(f"oracle quant_act_t_e8m0: bad sizes {M}x{K}")
+    return qt, st
+
+
+def quant_weight_e8m0(w_bf16: np.ndarray, want_t: bool = False):
+    """W[N][K] -> (Q[N][K], S[N/128][K/128] uint8 E8M0 codes, Q^T[K][N] or None)."""
+    w = _u16(w_bf16)
+    N, K = w.shape
+    q = np.empty((N, K), dtype=np.uint8)
+    s = np.empty((N // 128, K // 128), dtype=np.uint8)
+    qt = np.empty((K, N), dtype=np.uint8) if want_t else None
+    if _load().fp8o_quant_weight_e8m0(_ptr(w), N, K, _ptr(q), _ptr(s),
+                                      _ptr(qt) if want_t else None):
+        raise ValueError(f"oracle quant_weight_e8m0: bad sizes {N}x{K}")
     return q, s, qt
 
 

@@ -192,6 +192,113 @@ int fp8o_quant_weight(const uint16_t *w, int64_t N, int64_t K, uint8_t *q, float
     return 0;
 }
 
+/* ------------------------------------------------- power-of-two scales ---- */
+/*
+ * Section 3.2 of the same page: on the RTX 5090 the recipe's 128-blocks run through
+ * Transformer Engine's MXFP8 path, where every block scale is a power of two stored
+ * as an 8-bit exponent (E8M0).  Reading taken here: the scale of a group is the
+ * smallest power of two 2^e with amax <= 448 * 2^e (no value saturates), e clamped to
+ * [-127, 127], the E8M0 code being e + 127; an all-zero group takes e = -127 and
+ * codes 0x00.  Dividing by 2^e is exact, so each code is the single round-to-
+ * nearest-even of x * 2^-e onto E4M3.
+ */
+
+int fp8o_e8m0_exponent(float amax)
+{
+    if (!(amax > 0.0f))
+        return -127;
+    int E;
+    frexp((double)amax, &E);          /* amax = m * 2^E, m in [0.5, 1) */
+    int e = E - 10;                   /* 448 * 2^(E-10) < 2^(E-1) <= amax */
+    if (e < -127)
+        e = -127;
+    while ((double)amax > ldexp(448.0, e))
+        ++e;
+    return e > 127 ? 127 : e;
+}
+
+/* One group with a power-of-two scale: codes at q[i*qstride], returns the E8M0 code. */
+uint8_t fp8o_quantize_group_e8m0(const uint16_t *x, int64_t xstride, int64_t n,
+                                 uint8_t *q, int64_t qstride)
+{
+    float amax = 0.0f;
+    for (int64_t i = 0; i < n; ++i) {
+        float a = fabsf(bf16_to_float(x[i * xstride]));
+        if (a > amax)
+            amax = a;
+    }
+    if (amax == 0.0f) {
+        for (int64_t i = 0; i < n; ++i)
+            q[i * qstride] = 0x00;
+        return 0;
+    }
+    int e = fp8o_e8m0_exponent(amax);
+    for (int64_t i = 0; i < n; ++i) {
+        double v = ldexp((double)bf16_to_float(x[i * xstride]), -e);  /* exact */
+        q[i * qstride] = fp8o_e4m3_encode((float)v);
+    }
+    return (uint8_t)(e + 127);
+}
+
+int fp8o_quant_act_e8m0(const uint16_t *x, int64_t M, int64_t K, uint8_t *q, uint8_t *s)
+{
+    if (bad_sizes(M, K))
+        return -1;
+    int64_t KB = K / 128;
+#pragma omp parallel for schedule(static)
+    for (int64_t m = 0; m < M; ++m)
+        for (int64_t kb = 0; kb < KB; ++kb)
+            s[kb * M + m] = fp8o_quantize_group_e8m0(x + m * K + kb * 128, 1, 128,
+                                                     q + m * K + kb * 128, 1);
+    return 0;
+}
+
+int fp8o_quant_act_t_e8m0(const uint16_t *x, int64_t M, int64_t K, uint8_t *qt, uint8_t *st)
+{
+    if (bad_sizes(M, K))
+        return -1;
+    int64_t MB = M / 128;
+#pragma omp parallel for schedule(static)
+    for (int64_t k = 0; k < K; ++k)
+        for (int64_t mb = 0; mb < MB; ++mb)
+            st[mb * K + k] = fp8o_quantize_group_e8m0(x + mb * 128 * K + k, K, 128,
+                                                      qt + k * M + mb * 128, 1);
+    return 0;
+}
+
+int fp8o_quant_weight_e8m0(const uint16_t *w, int64_t N, int64_t K, uint8_t *q, uint8_t *s,
+                           uint8_t *qt_or_null)
+{
+    if (bad_sizes(N, K))
+        return -1;
+    int64_t NB = N / 128, KB = K / 128;
+#pragma omp parallel for schedule(static)
+    for (int64_t blk = 0; blk < NB * KB; ++blk) {
+        int64_t nb = blk / KB, kb = blk % KB;
+        const uint16_t *wb = w + nb * 128 * K + kb * 128;
+        float amax = 0.0f;
+        for (int64_t i = 0; i < 128; ++i)
+            for (int64_t j = 0; j < 128; ++j) {
+                float a = fabsf(bf16_to_float(wb[i * K + j]));
+                if (a > amax)
+                    amax = a;
+            }
+        int e = fp8o_e8m0_exponent(amax);
+        for (int64_t i = 0; i < 128; ++i)
+            for (int64_t j = 0; j < 128; ++j) {
+                int64_t n = nb * 128 + i, k = kb * 128 + j;
+                uint8_t code = 0x00;
+                if (amax != 0.0f)
+                    code = fp8o_e4m3_encode((float)ldexp((double)bf16_to_float(w[n * K + k]), -e));
+                q[n * K + k] = code;
+                if (qt_or_null)
+                    qt_or_null[k * N + n] = code;
+            }
+        s[nb * KB + kb] = (uint8_t)(amax != 0.0f ? e + 127 : 0);
+    }
+    return 0;
+}
+
 /* ---------------------------------------------------------------- GEMM ---- */
 
 /* Decoded value of every code, filled from fp8o_e4m3_decode before any

@@ -60,6 +60,18 @@ int fp8o_quant_act_t(const uint16_t *x, int64_t M, int64_t K, uint8_t *qt, float
 int fp8o_quant_weight(const uint16_t *w, int64_t N, int64_t K, uint8_t *q, float *s,
                       uint8_t *qt_or_null);
 
+/* Power-of-two (E8M0) scales, the MXFP8 form the same section says the recipe runs
+ * on its GPUs: the group scale is the smallest 2^e with amax <= 448 * 2^e, e in
+ * [-127, 127], stored as the code e + 127 (0 for an all-zero group, whose codes are
+ * 0x00); each value's code is RNE(x * 2^-e) onto E4M3 (no saturation occurs). */
+int fp8o_e8m0_exponent(float amax);
+uint8_t fp8o_quantize_group_e8m0(const uint16_t *x, int64_t xstride, int64_t n,
+                                 uint8_t *q, int64_t qstride);
+int fp8o_quant_act_e8m0(const uint16_t *x, int64_t M, int64_t K, uint8_t *q, uint8_t *s);
+int fp8o_quant_act_t_e8m0(const uint16_t *x, int64_t M, int64_t K, uint8_t *qt, uint8_t *st);
+int fp8o_quant_weight_e8m0(const uint16_t *w, int64_t N, int64_t K, uint8_t *q, uint8_t *s,
+                           uint8_t *qt_or_null);
+
 /* Modes of the blockwise GEMM, all producing D[M][N] summed over a reduction of
  * length K with one (a-scale x b-scale) pair per 128-long reduction block:
  *   0 FPROP: a[M][K] sa[K/128][M]; b[N][K] sb[N/128][K/128]      (Y  = X  . W^T)
