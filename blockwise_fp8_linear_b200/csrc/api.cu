@@ -159,6 +159,55 @@ int fp8_quant_weight(const void *w_bf16, int64_t N, int64_t K, uint8_t *q, float
                                                 static_cast<cudaStream_t>(stream)));
 }
 
+// ---- power-of-two (E8M0) scale variants: same layouts, uint8 scale codes ----
+
+static int quant_e8m0(int which, const void *x, int64_t M, int64_t K, uint8_t *q, uint8_t *s,
+                      uint8_t *qt, uint8_t *st, void *stream)
+{
+    if (!dim_ok(M) || !dim_ok(K))
+        return FP8BW_ESHAPE;
+    if (!aligned16(x) || (q && !aligned16(q)) || (s && !aligned16(s)) ||
+        (qt && !aligned16(qt)) || (st && !aligned16(st)))
+        return FP8BW_EALIGN;
+    int status;
+    if (device_sms({x, q, s, qt, st}, &status) < 0)
+        return status;
+    return from_cuda(fp8bw::launch_quant_e8m0(which, x, M, K, q, s, qt, st,
+                                              static_cast<cudaStream_t>(stream)));
+}
+
+int fp8_quant_act_e8m0(const void *x_bf16, int64_t M, int64_t K, uint8_t *q, uint8_t *s_e8m0,
+                       void *stream)
+{
+    if (!x_bf16 || !q || !s_e8m0)
+        return FP8BW_EINVAL;
+    return quant_e8m0(0, x_bf16, M, K, q, s_e8m0, nullptr, nullptr, stream);
+}
+
+int fp8_quant_act_t_e8m0(const void *x_bf16, int64_t M, int64_t K, uint8_t *qt,
+                         uint8_t *st_e8m0, void *stream)
+{
+    if (!x_bf16 || !qt || !st_e8m0)
+        return FP8BW_EINVAL;
+    return quant_e8m0(1, x_bf16, M, K, nullptr, nullptr, qt, st_e8m0, stream);
+}
+
+int fp8_quant_act_dual_e8m0(const void *x_bf16, int64_t M, int64_t K, uint8_t *q,
+                            uint8_t *s_e8m0, uint8_t *qt, uint8_t *st_e8m0, void *stream)
+{
+    if (!x_bf16 || !q || !s_e8m0 || !qt || !st_e8m0)
+        return FP8BW_EINVAL;
+    return quant_e8m0(2, x_bf16, M, K, q, s_e8m0, qt, st_e8m0, stream);
+}
+
+int fp8_quant_weight_e8m0(const void *w_bf16, int64_t N, int64_t K, uint8_t *q,
+                          uint8_t *s_e8m0, uint8_t *qt_or_null, void *stream)
+{
+    if (!w_bf16 || !q || !s_e8m0)
+        return FP8BW_EINVAL;
+    return quant_e8m0(3, w_bf16, N, K, q, s_e8m0, qt_or_null, nullptr, stream);
+}
+
 int fp8_gemm_blockwise(int mode, const uint8_t *a, const float *sa, const uint8_t *b,
                        const float *sb, void *d_bf16, int64_t M, int64_t N, int64_t K,
                        void *stream)

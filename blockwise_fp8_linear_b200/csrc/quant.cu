@@ -92,6 +92,42 @@ __device__ __forceinline__ uint2 quant8(uint4 v, const GroupDiv &d)
     return make_uint2(c[0] | (c[1] << 16), c[2] | (c[3] << 16));
 }
 
+// Power-of-two (E8M0) scales, the MXFP8 form of the recipe (same section): the group
+// scale is the smallest 2^e with amax <= 448 * 2^e, e clamped to [-127, 127] (a zero
+// or subnormal amax gives -127), stored as the code e + 127.  amax = m * 2^E with
+// m in [1, 2): 448 * 2^(E-8) = 1.75 * 2^E >= amax exactly when m <= 1.75, else one
+// more power is needed.  Multiplying by 2^-e is exact, so each value's code is a
+// single rounding of x * 2^-e onto E4M3 (never saturating).
+__device__ __forceinline__ int e8m0_exponent(float amax)
+{
+    const uint32_t b = __float_as_uint(amax);
+    const int be = int(b >> 23);
+    if (be == 0)
+        return -127;
+    const int e = be - 135 + ((b & 0x7FFFFFu) > 0x600000u ? 1 : 0);
+    return e < -127 ? -127 : (e > 126 ? 126 : e);
+}
+
+// 2^-e as a float (e in [-127, 126]).
+__device__ __forceinline__ float pow2_neg(int e)
+{
+    return __uint_as_float(uint32_t(127 - e) << 23);
+}
+
+// Eight BF16 values of one group times the power of two `mul` -> eight E4M3 codes.
+__device__ __forceinline__ uint2 quant8_pow2(uint4 v, float mul)
+{
+    const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+    const float2 m2 = make_float2(mul, mul);
+    uint32_t c[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        const float2 q = __fmul2_rn(make_float2(bf16lo(w[i]), bf16hi(w[i])), m2);
+        c[i] = cvt_e4m3x2(q.x, q.y);
+    }
+    return make_uint2(c[0] | (c[1] << 16), c[2] | (c[3] << 16));
+}
+
 // ------------------------------------------------------------ fp8_quant_act
 
 // A warp quantizes two consecutive groups at a time (half-warp h takes group
@@ -232,9 +268,11 @@ quant_act_t_kernel(const uint32_t *__restrict__ x, int64_t M, int64_t K,
 // pass*16 + t/16 and columns (t%16)*8 .. +7.
 constexpr int QW_THREADS = 256;
 
+// E8: power-of-two scales, s is uint8_t[N/128][K/128] of E8M0 codes.
+template <bool E8>
 __global__ void __launch_bounds__(QW_THREADS)
 quant_weight_kernel(const uint4 *__restrict__ w, int64_t N, int64_t K, uint2 *__restrict__ q,
-                    float *__restrict__ s, uint8_t *__restrict__ qt)
+                    void *__restrict__ s_out, uint8_t *__restrict__ qt)
 {
     __shared__ uint32_t red[8];
     __shared__ uint8_t tile[128][144];  // codes, for the optional transposed copy
@@ -262,7 +300,8 @@ quant_weight_kernel(const uint4 *__restrict__ w, int64_t N, int64_t K, uint2 *__
     for (int i = 0; i < 8; ++i)
         m2 = __vmaxu2(m2, red[i]);
     const float amax = halves_max_to_float(m2);
-    const float sc = __fdiv_rn(amax, 448.0f);
+    const float sc = E8 ? 0.0f : __fdiv_rn(amax, 448.0f);
+    const int e = E8 ? e8m0_exponent(amax) : 0;
     const GroupDiv div(sc);
 
 #pragma unroll
@@ -270,13 +309,17 @@ quant_weight_kernel(const uint4 *__restrict__ w, int64_t N, int64_t K, uint2 *__
         int64_t n = nb * 128 + p * 16 + rsub;
         uint2 c = make_uint2(0u, 0u);
         if (amax != 0.0f)
-            c = quant8(v[p], div);
+            c = E8 ? quant8_pow2(v[p], pow2_neg(e)) : quant8(v[p], div);
         q[(n * K + kb * 128 + csub) / 8] = c;
         if (qt)
             *reinterpret_cast<uint2 *>(&tile[p * 16 + rsub][csub]) = c;
     }
-    if (t == 0)
-        s[nb * (K / 128) + kb] = sc;
+    if (t == 0) {
+        if (E8)
+            static_cast<uint8_t *>(s_out)[nb * (K / 128) + kb] = amax != 0.0f ? uint8_t(e + 127) : 0;
+        else
+            static_cast<float *>(s_out)[nb * (K / 128) + kb] = sc;
+    }
     if (qt) {
         __syncthreads();
         // qt[k][n]: thread t writes column k = t/2 of the block, 64 rows starting at
@@ -311,10 +354,11 @@ quant_weight_kernel(const uint4 *__restrict__ w, int64_t N, int64_t K, uint2 *__
 // With both, X is read once for the two layouts wgrad and fprop/dgrad need.
 constexpr int QD_THREADS = 256;
 
-template <bool ROWS, bool COLS>
+// E8: power-of-two scales; s and st are then uint8_t arrays of E8M0 codes.
+template <bool ROWS, bool COLS, bool E8 = false>
 __global__ void __launch_bounds__(QD_THREADS)
 quant_tile_kernel(const uint4 *__restrict__ x, int64_t M, int64_t K, uint2 *__restrict__ q,
-                  float *__restrict__ s, uint8_t *__restrict__ qt, float *__restrict__ st)
+                  void *__restrict__ s_out, uint8_t *__restrict__ qt, void *__restrict__ st_out)
 {
     __shared__ uint32_t tile[COLS ? 128 * 64 : 1];
     __shared__ uint32_t red[4][64];
@@ -337,14 +381,22 @@ quant_tile_kernel(const uint4 *__restrict__ x, int64_t M, int64_t K, uint2 *__re
             for (int o = 8; o >= 1; o >>= 1)
                 m2 = __vmaxu2(m2, __shfl_xor_sync(0xffffffffu, m2, o));
             const float amax = halves_max_to_float(m2);
-            const float sc = __fdiv_rn(amax, 448.0f);
-            uint2 codes = make_uint2(0u, 0u);
-            if (amax != 0.0f)
-                codes = quant8(v[p], GroupDiv(sc));
             const int64_t m = mb * 128 + row;
+            uint2 codes = make_uint2(0u, 0u);
+            if constexpr (E8) {
+                const int e = e8m0_exponent(amax);
+                if (amax != 0.0f)
+                    codes = quant8_pow2(v[p], pow2_neg(e));
+                if (sub == 0)
+                    static_cast<uint8_t *>(s_out)[kb * M + m] = amax != 0.0f ? uint8_t(e + 127) : 0;
+            } else {
+                const float sc = __fdiv_rn(amax, 448.0f);
+                if (amax != 0.0f)
+                    codes = quant8(v[p], GroupDiv(sc));
+                if (sub == 0)
+                    static_cast<float *>(s_out)[kb * M + m] = sc;
+            }
             q[(m * K + kb * 128) / 8 + sub] = codes;
-            if (sub == 0)
-                s[kb * M + m] = sc;
         }
         if (COLS)
             *reinterpret_cast<uint4 *>(&tile[row * 64 + sub * 4]) = v[p];
@@ -365,14 +417,25 @@ quant_tile_kernel(const uint4 *__restrict__ x, int64_t M, int64_t K, uint2 *__re
         m2 = __vmaxu2(__vmaxu2(red[0][cp], red[1][cp]), __vmaxu2(red[2][cp], red[3][cp]));
         const float amax_lo = __uint_as_float((m2 & 0xFFFFu) << 16);
         const float amax_hi = __uint_as_float(m2 & 0xFFFF0000u);
-        const float s_lo = __fdiv_rn(amax_lo, 448.0f);
-        const float s_hi = __fdiv_rn(amax_hi, 448.0f);
+        const float s_lo = E8 ? 0.0f : __fdiv_rn(amax_lo, 448.0f);
+        const float s_hi = E8 ? 0.0f : __fdiv_rn(amax_hi, 448.0f);
+        const int e_lo = E8 ? e8m0_exponent(amax_lo) : 0;
+        const int e_hi = E8 ? e8m0_exponent(amax_hi) : 0;
         uint32_t clo[8], chi[8];
 #pragma unroll
         for (int i = 0; i < 8; ++i)
             clo[i] = chi[i] = 0u;
         const GroupDiv dlo(s_lo), dhi(s_hi);
-        if (dlo.fast && dhi.fast) {
+        if (E8) {
+            const float2 mul2 = make_float2(pow2_neg(e_lo), pow2_neg(e_hi));
+#pragma unroll
+            for (int i = 0; i < 32; i += 2) {
+                const float2 a = __fmul2_rn(make_float2(bf16lo(w[i]), bf16hi(w[i])), mul2);
+                const float2 b = __fmul2_rn(make_float2(bf16lo(w[i + 1]), bf16hi(w[i + 1])), mul2);
+                clo[i / 4] |= cvt_e4m3x2(a.x, b.x) << (16 * ((i / 2) & 1));
+                chi[i / 4] |= cvt_e4m3x2(a.y, b.y) << (16 * ((i / 2) & 1));
+            }
+        } else if (dlo.fast && dhi.fast) {
             const float2 r2 = make_float2(dlo.r, dhi.r), ns2 = make_float2(-s_lo, -s_hi);
 #pragma unroll
             for (int i = 0; i < 32; i += 2) {
@@ -410,8 +473,14 @@ quant_tile_kernel(const uint4 *__restrict__ x, int64_t M, int64_t K, uint2 *__re
         dlo_p[1] = make_uint4(clo[4], clo[5], clo[6], clo[7]);
         dhi_p[0] = make_uint4(chi[0], chi[1], chi[2], chi[3]);
         dhi_p[1] = make_uint4(chi[4], chi[5], chi[6], chi[7]);
-        if (rq == 0)
-            *reinterpret_cast<float2 *>(st + mb * K + col) = make_float2(s_lo, s_hi);
+        if (rq == 0) {
+            if (E8)
+                *reinterpret_cast<uint16_t *>(static_cast<uint8_t *>(st_out) + mb * K + col) =
+                    uint16_t((amax_lo != 0.0f ? e_lo + 127 : 0) | ((amax_hi != 0.0f ? e_hi + 127 : 0) << 8));
+            else
+                *reinterpret_cast<float2 *>(static_cast<float *>(st_out) + mb * K + col) =
+                    make_float2(s_lo, s_hi);
+        }
     }
 }
 
@@ -470,8 +539,35 @@ cudaError_t launch_quant_weight(const void *w, int64_t N, int64_t K, uint8_t *q,
                                 uint8_t *qt, cudaStream_t stream)
 {
     dim3 grid(unsigned(K / 128), unsigned(N / 128));
-    quant_weight_kernel<<<grid, QW_THREADS, 0, stream>>>(
+    quant_weight_kernel<false><<<grid, QW_THREADS, 0, stream>>>(
         static_cast<const uint4 *>(w), N, K, reinterpret_cast<uint2 *>(q), s, qt);
+    return cudaGetLastError();
+}
+
+// Power-of-two (E8M0) scale quantizers: the same layouts with uint8 scale codes.
+cudaError_t launch_quant_e8m0(int which, const void *x, int64_t M, int64_t K, uint8_t *q,
+                              uint8_t *s, uint8_t *qt, uint8_t *st, cudaStream_t stream)
+{
+    dim3 grid(unsigned(K / 128), unsigned(M / 128));
+    const uint4 *xv = static_cast<const uint4 *>(x);
+    uint2 *qv = reinterpret_cast<uint2 *>(q);
+    switch (which) {
+    case 0:  // rows: q[M][K], s[K/128][M]
+        quant_tile_kernel<true, false, true><<<grid, QD_THREADS, 0, stream>>>(xv, M, K, qv, s,
+                                                                            nullptr, nullptr);
+        break;
+    case 1:  // token groups: qt[K][M], st[M/128][K]
+        quant_tile_kernel<false, true, true><<<grid, QD_THREADS, 0, stream>>>(xv, M, K, nullptr,
+                                                                            nullptr, qt, st);
+        break;
+    case 2:  // both
+        quant_tile_kernel<true, true, true><<<grid, QD_THREADS, 0, stream>>>(xv, M, K, qv, s, qt,
+                                                                           st);
+        break;
+    default:  // weight blocks: q[N=M][K], s[M/128][K/128], optional qt[K][M]
+        quant_weight_kernel<true><<<grid, QW_THREADS, 0, stream>>>(xv, M, K, qv, s, qt);
+        break;
+    }
     return cudaGetLastError();
 }
 

@@ -12,6 +12,11 @@ cudaError_t launch_quant_act_t(const void *x, int64_t M, int64_t K, uint8_t *qt,
                                cudaStream_t stream);
 cudaError_t launch_quant_dual(const void *x, int64_t M, int64_t K, uint8_t *q, float *s,
                               uint8_t *qt, float *st, cudaStream_t stream);
+// Power-of-two (E8M0) scale quantizers (which: 0 rows, 1 token groups, 2 both,
+// 3 weight blocks with rows = M); scales are uint8 E8M0 codes in the FP32 layouts.
+cudaError_t launch_quant_e8m0(int which, const void *x, int64_t M, int64_t K, uint8_t *q,
+                              uint8_t *s, uint8_t *qt, uint8_t *st, cudaStream_t stream);
+
 cudaError_t launch_quant_weight(const void *w, int64_t N, int64_t K, uint8_t *q, float *s,
                                 uint8_t *qt, cudaStream_t stream);
 
