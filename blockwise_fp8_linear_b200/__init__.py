@@ -21,6 +21,8 @@ __all__ = [
     "FPROP", "DGRAD", "WGRAD", "Fp8bwError", "lib", "library_path",
     "fp8_quant_act", "fp8_quant_act_t", "fp8_quant_act_dual", "fp8_quant_weight",
     "fp8_gemm_blockwise", "fp8_gemm_wgrad_acc32",
+    "fp8_quant_act_e8m0", "fp8_quant_act_t_e8m0", "fp8_quant_act_dual_e8m0",
+    "fp8_quant_weight_e8m0", "fp8_gemm_blockwise_e8m0",
     "fp8bw_status_string", "fp8bw_last_device_error", "fp8bw_version",
     "fp8bw_selftest_wait_timeout",
     "linear_fprop", "linear_dgrad", "linear_wgrad",
@@ -55,8 +57,15 @@ def lib():
         L.fp8_quant_weight.argtypes = [vp, i64, i64, vp, vp, vp, vp]
         L.fp8_gemm_blockwise.argtypes = [i32, vp, vp, vp, vp, vp, i64, i64, i64, vp]
         L.fp8_gemm_wgrad_acc32.argtypes = [vp, vp, vp, vp, vp, i64, i64, i64, vp]
+        L.fp8_quant_act_e8m0.argtypes = [vp, i64, i64, vp, vp, vp]
+        L.fp8_quant_act_t_e8m0.argtypes = [vp, i64, i64, vp, vp, vp]
+        L.fp8_quant_act_dual_e8m0.argtypes = [vp, i64, i64, vp, vp, vp, vp, vp]
+        L.fp8_quant_weight_e8m0.argtypes = [vp, i64, i64, vp, vp, vp, vp]
+        L.fp8_gemm_blockwise_e8m0.argtypes = [i32, vp, vp, vp, vp, vp, i64, i64, i64, vp]
         for f in (L.fp8_quant_act, L.fp8_quant_act_t, L.fp8_quant_act_dual, L.fp8_quant_weight,
-                  L.fp8_gemm_blockwise, L.fp8_gemm_wgrad_acc32):
+                  L.fp8_gemm_blockwise, L.fp8_gemm_wgrad_acc32, L.fp8_quant_act_e8m0,
+                  L.fp8_quant_act_t_e8m0, L.fp8_quant_act_dual_e8m0, L.fp8_quant_weight_e8m0,
+                  L.fp8_gemm_blockwise_e8m0):
             f.restype = i32
         L.fp8bw_status_string.argtypes = [i32]
         L.fp8bw_status_string.restype = C.c_char_p
@@ -190,6 +199,78 @@ def fp8_gemm_wgrad_acc32(a, sa, b, sb, M: int, N: int, K: int, dw32, stream=None
                                       dw32.data_ptr(), M, N, K, _stream(stream)),
            "fp8_gemm_wgrad_acc32")
     return dw32
+
+
+# -- power-of-two (E8M0) scales: the MXFP8 form of the recipe --------------------
+
+def fp8_quant_act_e8m0(x, q=None, s=None, stream=None):
+    """X[M][K] bf16 -> (Q[M][K] uint8, S: E8M0 scale blocks [M/128][(K/128)*512] uint8,
+    the tensor-core layout described in include/fp8bw.h)."""
+    import torch
+    _need(x, torch.bfloat16, 2, "x")
+    M, K = x.shape
+    q = torch.empty((M, K), dtype=torch.uint8, device=x.device) if q is None else q
+    s = torch.empty((M // 128, (K // 128) * 512), dtype=torch.uint8, device=x.device) if s is None else s
+    _check(lib().fp8_quant_act_e8m0(x.data_ptr(), M, K, q.data_ptr(), s.data_ptr(),
+                                    _stream(stream)), "fp8_quant_act_e8m0")
+    return q, s
+
+
+def fp8_quant_act_t_e8m0(x, qt=None, st=None, stream=None):
+    """X[M][K] bf16 -> (Q^T[K][M] uint8, S^T: E8M0 scale blocks [K/128][(M/128)*512])."""
+    import torch
+    _need(x, torch.bfloat16, 2, "x")
+    M, K = x.shape
+    qt = torch.empty((K, M), dtype=torch.uint8, device=x.device) if qt is None else qt
+    st = torch.empty((K // 128, (M // 128) * 512), dtype=torch.uint8, device=x.device) if st is None else st
+    _check(lib().fp8_quant_act_t_e8m0(x.data_ptr(), M, K, qt.data_ptr(), st.data_ptr(),
+                                      _stream(stream)), "fp8_quant_act_t_e8m0")
+    return qt, st
+
+
+def fp8_quant_act_dual_e8m0(x, stream=None):
+    """X[M][K] bf16 -> (Q, S, Q^T, S^T) with E8M0 scale codes, from one read of X."""
+    import torch
+    _need(x, torch.bfloat16, 2, "x")
+    M, K = x.shape
+    dev = x.device
+    q = torch.empty((M, K), dtype=torch.uint8, device=dev)
+    s = torch.empty((M // 128, (K // 128) * 512), dtype=torch.uint8, device=dev)
+    qt = torch.empty((K, M), dtype=torch.uint8, device=dev)
+    st = torch.empty((K // 128, (M // 128) * 512), dtype=torch.uint8, device=dev)
+    _check(lib().fp8_quant_act_dual_e8m0(x.data_ptr(), M, K, q.data_ptr(), s.data_ptr(),
+                                         qt.data_ptr(), st.data_ptr(), _stream(stream)),
+           "fp8_quant_act_dual_e8m0")
+    return q, s, qt, st
+
+
+def fp8_quant_weight_e8m0(w, want_t: bool = False, stream=None):
+    """W[N][K] bf16 -> (Q[N][K], S: E8M0 scale blocks [N/128][(K/128)*512], Q^T or None)."""
+    import torch
+    _need(w, torch.bfloat16, 2, "w")
+    N, K = w.shape
+    q = torch.empty((N, K), dtype=torch.uint8, device=w.device)
+    s = torch.empty((N // 128, (K // 128) * 512), dtype=torch.uint8, device=w.device)
+    qt = torch.empty((K, N), dtype=torch.uint8, device=w.device) if want_t else None
+    _check(lib().fp8_quant_weight_e8m0(w.data_ptr(), N, K, q.data_ptr(), s.data_ptr(),
+                                       qt.data_ptr() if want_t else None, _stream(stream)),
+           "fp8_quant_weight_e8m0")
+    return q, s, qt
+
+
+def fp8_gemm_blockwise_e8m0(mode: int, a, sa, b, sb, M: int, N: int, K: int, out=None,
+                            stream=None):
+    """fp8_gemm_blockwise with E8M0 scale blocks (from the *_e8m0 quantizers), applied by
+    the block-scaled MMA."""
+    import torch
+    for t, dt, name in ((a, torch.uint8, "a"), (b, torch.uint8, "b"),
+                        (sa, torch.uint8, "sa"), (sb, torch.uint8, "sb")):
+        _need(t, dt, 2, name)
+    out = torch.empty((M, N), dtype=torch.bfloat16, device=a.device) if out is None else out
+    _check(lib().fp8_gemm_blockwise_e8m0(int(mode), a.data_ptr(), sa.data_ptr(), b.data_ptr(),
+                                         sb.data_ptr(), out.data_ptr(), M, N, K, _stream(stream)),
+           "fp8_gemm_blockwise_e8m0")
+    return out
 
 
 # -- the three GEMMs of the linear layer, composed from the entry points above ----

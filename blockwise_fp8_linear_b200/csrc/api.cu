@@ -208,6 +208,25 @@ int fp8_quant_weight_e8m0(const void *w_bf16, int64_t N, int64_t K, uint8_t *q,
     return quant_e8m0(3, w_bf16, N, K, q, s_e8m0, qt_or_null, nullptr, stream);
 }
 
+int fp8_gemm_blockwise_e8m0(int mode, const uint8_t *a, const uint8_t *sa_e8m0,
+                            const uint8_t *b, const uint8_t *sb_e8m0, void *d_bf16, int64_t M,
+                            int64_t N, int64_t K, void *stream)
+{
+    if (mode < FP8BW_FPROP || mode > FP8BW_WGRAD || !a || !sa_e8m0 || !b || !sb_e8m0 || !d_bf16)
+        return FP8BW_EINVAL;
+    if (!dim_ok(M) || !dim_ok(N) || !dim_ok(K))
+        return FP8BW_ESHAPE;
+    if (!aligned16(a) || !aligned16(sa_e8m0) || !aligned16(b) || !aligned16(sb_e8m0) ||
+        !aligned16(d_bf16))
+        return FP8BW_EALIGN;
+    int st;
+    const int sms = device_sms({a, sa_e8m0, b, sb_e8m0, d_bf16}, &st);
+    if (sms < 0)
+        return st;
+    return from_cuda(fp8bw::launch_gemm_mx(mode, a, sa_e8m0, b, sb_e8m0, d_bf16, M, N, K,
+                                           static_cast<cudaStream_t>(stream), sms));
+}
+
 int fp8_gemm_blockwise(int mode, const uint8_t *a, const float *sa, const uint8_t *b,
                        const float *sb, void *d_bf16, int64_t M, int64_t N, int64_t K,
                        void *stream)
@@ -262,10 +281,11 @@ int fp8bw_last_device_error(void *stream)
     int st;
     if (device_sms({}, &st) < 0)
         return st;
-    int v = 0;
-    if (fp8bw::read_and_clear_device_error(static_cast<cudaStream_t>(stream), &v) != cudaSuccess)
+    int v = 0, w = 0;
+    if (fp8bw::read_and_clear_device_error(static_cast<cudaStream_t>(stream), &v) != cudaSuccess ||
+        fp8bw::read_and_clear_mx_error(&w) != cudaSuccess)
         return FP8BW_ECUDA;
-    return v ? FP8BW_ETIMEOUT : FP8BW_OK;
+    return (v || w) ? FP8BW_ETIMEOUT : FP8BW_OK;
 }
 
 int fp8bw_selftest_wait_timeout(int64_t limit_us, void *stream)

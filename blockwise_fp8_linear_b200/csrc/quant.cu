@@ -108,6 +108,16 @@ __device__ __forceinline__ int e8m0_exponent(float amax)
     return e < -127 ? -127 : (e > 126 ? 126 : e);
 }
 
+// E8M0 scales are stored in the layout the tensor cores read scale factors in: one
+// 512-byte block per 128 rows x 128-deep reduction block, in which the code of row r
+// fills bytes 16 (r % 32) + 4 (r / 32) .. +3 (repeated for the four 32-wide K steps).
+__device__ __forceinline__ uint32_t sf_block_off(int r) { return uint32_t((r & 31) * 16 + ((r >> 5) & 3) * 4); }
+
+__device__ __forceinline__ uint32_t rep4_code(int e, float amax)
+{
+    return amax != 0.0f ? uint32_t(e + 127) * 0x01010101u : 0u;
+}
+
 // 2^-e as a float (e in [-127, 126]).
 __device__ __forceinline__ float pow2_neg(int e)
 {
@@ -268,7 +278,8 @@ quant_act_t_kernel(const uint32_t *__restrict__ x, int64_t M, int64_t K,
 // pass*16 + t/16 and columns (t%16)*8 .. +7.
 constexpr int QW_THREADS = 256;
 
-// E8: power-of-two scales, s is uint8_t[N/128][K/128] of E8M0 codes.
+// E8: power-of-two scales, s is [N/128][K/128] blocks of 512 bytes, every byte of
+// block (nb, kb) the E8M0 code of that weight block.
 template <bool E8>
 __global__ void __launch_bounds__(QW_THREADS)
 quant_weight_kernel(const uint4 *__restrict__ w, int64_t N, int64_t K, uint2 *__restrict__ q,
@@ -314,11 +325,14 @@ quant_weight_kernel(const uint4 *__restrict__ w, int64_t N, int64_t K, uint2 *__
         if (qt)
             *reinterpret_cast<uint2 *>(&tile[p * 16 + rsub][csub]) = c;
     }
-    if (t == 0) {
-        if (E8)
-            static_cast<uint8_t *>(s_out)[nb * (K / 128) + kb] = amax != 0.0f ? uint8_t(e + 127) : 0;
-        else
-            static_cast<float *>(s_out)[nb * (K / 128) + kb] = sc;
+    if (E8) {
+        if (t < 32) {
+            const uint32_t w = rep4_code(e, amax);
+            reinterpret_cast<uint4 *>(static_cast<uint8_t *>(s_out) + (nb * (K / 128) + kb) * 512)[t] =
+                make_uint4(w, w, w, w);
+        }
+    } else if (t == 0) {
+        static_cast<float *>(s_out)[nb * (K / 128) + kb] = sc;
     }
     if (qt) {
         __syncthreads();
@@ -354,7 +368,9 @@ quant_weight_kernel(const uint4 *__restrict__ w, int64_t N, int64_t K, uint2 *__
 // With both, X is read once for the two layouts wgrad and fprop/dgrad need.
 constexpr int QD_THREADS = 256;
 
-// E8: power-of-two scales; s and st are then uint8_t arrays of E8M0 codes.
+// E8: power-of-two scales in 512-byte blocks (see sf_block_off): s holds
+// [M/128][K/128] blocks (row m of block (m/128, kb)), st holds [K/128][M/128] blocks
+// (column k of X is row k % 128 of block (k/128, mb)).
 template <bool ROWS, bool COLS, bool E8 = false>
 __global__ void __launch_bounds__(QD_THREADS)
 quant_tile_kernel(const uint4 *__restrict__ x, int64_t M, int64_t K, uint2 *__restrict__ q,
@@ -388,7 +404,9 @@ quant_tile_kernel(const uint4 *__restrict__ x, int64_t M, int64_t K, uint2 *__re
                 if (amax != 0.0f)
                     codes = quant8_pow2(v[p], pow2_neg(e));
                 if (sub == 0)
-                    static_cast<uint8_t *>(s_out)[kb * M + m] = amax != 0.0f ? uint8_t(e + 127) : 0;
+                    *reinterpret_cast<uint32_t *>(static_cast<uint8_t *>(s_out) +
+                                                  ((m >> 7) * (K / 128) + kb) * 512 + sf_block_off(int(m & 127))) =
+                        rep4_code(e, amax);
             } else {
                 const float sc = __fdiv_rn(amax, 448.0f);
                 if (amax != 0.0f)
@@ -474,10 +492,11 @@ quant_tile_kernel(const uint4 *__restrict__ x, int64_t M, int64_t K, uint2 *__re
         dhi_p[0] = make_uint4(chi[0], chi[1], chi[2], chi[3]);
         dhi_p[1] = make_uint4(chi[4], chi[5], chi[6], chi[7]);
         if (rq == 0) {
-            if (E8)
-                *reinterpret_cast<uint16_t *>(static_cast<uint8_t *>(st_out) + mb * K + col) =
-                    uint16_t((amax_lo != 0.0f ? e_lo + 127 : 0) | ((amax_hi != 0.0f ? e_hi + 127 : 0) << 8));
-            else
+            if (E8) {
+                uint8_t *blk = static_cast<uint8_t *>(st_out) + ((col >> 7) * (M / 128) + mb) * 512;
+                *reinterpret_cast<uint32_t *>(blk + sf_block_off(int(col & 127))) = rep4_code(e_lo, amax_lo);
+                *reinterpret_cast<uint32_t *>(blk + sf_block_off(int((col + 1) & 127))) = rep4_code(e_hi, amax_hi);
+            } else
                 *reinterpret_cast<float2 *>(static_cast<float *>(st_out) + mb * K + col) =
                     make_float2(s_lo, s_hi);
         }
@@ -544,7 +563,8 @@ cudaError_t launch_quant_weight(const void *w, int64_t N, int64_t K, uint8_t *q,
     return cudaGetLastError();
 }
 
-// Power-of-two (E8M0) scale quantizers: the same layouts with uint8 scale codes.
+// Power-of-two (E8M0) scale quantizers: the same code layouts, scales as 512-byte
+// tensor-core scale blocks.
 cudaError_t launch_quant_e8m0(int which, const void *x, int64_t M, int64_t K, uint8_t *q,
                               uint8_t *s, uint8_t *qt, uint8_t *st, cudaStream_t stream)
 {

@@ -31,6 +31,15 @@ cudaError_t launch_gemm_wgrad_acc32(const uint8_t *a, const float *sa, const uin
                                     const float *sb, float *d32, int64_t M, int64_t N, int64_t K,
                                     cudaStream_t stream, int num_sms);
 
+// GEMM with power-of-two (E8M0) scale codes (uint8, the layouts of the FP32 scales),
+// promoted inside the block-scaled MMA.  Arguments already validated.
+cudaError_t launch_gemm_mx(int mode, const uint8_t *a, const uint8_t *sa, const uint8_t *b,
+                           const uint8_t *sb, void *d, int64_t M, int64_t N, int64_t K,
+                           cudaStream_t stream, int num_sms);
+
+// Error word of the E8M0 GEMM's bounded waits (read and cleared; caller synchronizes).
+cudaError_t read_and_clear_mx_error(int *value);
+
 // Bounded-wait self-test (records a timeout in the error word, no fault).
 cudaError_t launch_selftest_wait(uint64_t limit_ns, cudaStream_t stream);
 

@@ -146,6 +146,53 @@ int fp8_gemm_blockwise(int mode, const uint8_t *a, const float *sa, const uint8_
 int fp8_gemm_wgrad_acc32(const uint8_t *a, const float *sa, const uint8_t *b, const float *sb,
                          float *dw32, int64_t M, int64_t N, int64_t K, void *stream);
 
+/*
+ * ---- Power-of-two (E8M0) scales: the MXFP8 form of the recipe ----
+ * Section 3.2: on the RTX 5090 the 128-blocks run through Transformer Engine's MXFP8
+ * path, where every block scale is a power of two stored as an 8-bit exponent.
+ * These entry points keep the groupings and code layouts above; each scale is the
+ * E8M0 code e + 127 of 2^e, the smallest power of two with amax <= 448 * 2^e (e
+ * clamped to [-127, 127]), and each value's code is the round-to-nearest-even of
+ * x * 2^-e onto E4M3, which never saturates.  An all-zero group gets code 0 and
+ * codes 0x00.
+ *
+ * Scale layout (the one the tensor cores read scale factors in): 512-byte blocks, one
+ * per 128 rows x 128-deep reduction block; in a block the code of row r (0..127)
+ * fills bytes 16 (r % 32) + 4 (r / 32) .. +3 (the code repeated four times, once per
+ * 32-wide K step of the MMA).
+ *   fp8_quant_act_e8m0       x[M][K] -> q[M][K]; s: [M/128][K/128] blocks, rows m
+ *   fp8_quant_act_t_e8m0     x[M][K] -> qt[K][M]; st: [K/128][M/128] blocks, the
+ *                            columns k of x as rows (the wgrad operand's rows)
+ *   fp8_quant_act_dual_e8m0  both, from one read of x
+ *   fp8_quant_weight_e8m0    w[N][K] -> q[N][K]; s: [N/128][K/128] blocks, every byte
+ *                            of block (nb, kb) the code of that weight block;
+ *                            optional qt[K][N]
+ * Buffer sizes: M*K/32 bytes of scales for the activation forms, N*K/32 for the
+ * weight.  Errors and pointer rules as above (every pointer 16-byte aligned).
+ */
+int fp8_quant_act_e8m0(const void *x_bf16, int64_t M, int64_t K, uint8_t *q, uint8_t *s_e8m0,
+                       void *stream);
+int fp8_quant_act_t_e8m0(const void *x_bf16, int64_t M, int64_t K, uint8_t *qt,
+                         uint8_t *st_e8m0, void *stream);
+int fp8_quant_act_dual_e8m0(const void *x_bf16, int64_t M, int64_t K, uint8_t *q,
+                            uint8_t *s_e8m0, uint8_t *qt, uint8_t *st_e8m0, void *stream);
+int fp8_quant_weight_e8m0(const void *w_bf16, int64_t N, int64_t K, uint8_t *q,
+                          uint8_t *s_e8m0, uint8_t *qt_or_null, void *stream);
+
+/*
+ * fp8_gemm_blockwise_e8m0 -- fp8_gemm_blockwise with E8M0 scales (same modes and
+ * operand layouts; sa / sb the scale blocks above: FPROP sa from fp8_quant_act_e8m0,
+ * sb from fp8_quant_weight_e8m0; DGRAD the same weight blocks, read transposed;
+ * WGRAD both from fp8_quant_act_t_e8m0).  The scales are applied
+ * by the tensor cores (tcgen05.mma kind::mxf8f6f4.block_scale, each 128-block's
+ * scale repeated over its four 32-wide K steps), so the reduction accumulates in one
+ * FP32 accumulator and the result is rounded to BF16 once: D = sum_k
+ * (qa 2^ea)(qb 2^eb).  d_bf16 [M][N] is written, never read.
+ */
+int fp8_gemm_blockwise_e8m0(int mode, const uint8_t *a, const uint8_t *sa_e8m0,
+                            const uint8_t *b, const uint8_t *sb_e8m0, void *d_bf16, int64_t M,
+                            int64_t N, int64_t K, void *stream);
+
 /* Human-readable name of a status code (static string). */
 const char *fp8bw_status_string(int status);
 

@@ -65,6 +65,13 @@ def test_argument_errors_before_any_launch(L):
     assert L.fp8_quant_act_dual(p, 128, 100, p, p, p, p, s) == 3
     assert L.fp8_gemm_wgrad_acc32(p, p, p, p, nul, 128, 128, 128, s) == 1
     assert L.fp8_gemm_wgrad_acc32(p, p, p, p, odd, 128, 128, 128, s) == 2
+    assert L.fp8_quant_act_e8m0(nul, 128, 128, p, p, s) == 1
+    assert L.fp8_quant_act_t_e8m0(p, 128, 200, p, p, s) == 3
+    assert L.fp8_quant_act_dual_e8m0(p, 128, 128, p, p, p, odd, s) == 2
+    assert L.fp8_quant_weight_e8m0(p, 128, 128, p, nul, nul, s) == 1
+    assert L.fp8_gemm_blockwise_e8m0(5, p, p, p, p, p, 128, 128, 128, s) == 1
+    assert L.fp8_gemm_blockwise_e8m0(2, p, p, p, p, p, 128, 128, 130, s) == 3
+    assert L.fp8_gemm_blockwise_e8m0(0, p, odd, p, p, p, 128, 128, 128, s) == 2
 
 
 def test_no_gpu_reports_cuda_error_not_crash(L):
