@@ -14,6 +14,10 @@ that the SMs one GEMM leaves idle in its last round of tiles take the other's
 the 12 GEMMs, divided by the time of all quantizers and GEMMs); the kernel roofline
 comes from a separate one-stream pass with every GEMM bracketed by events.
 
+The line also carries "variant_e8m0": the same step with power-of-two (E8M0) scales,
+applied by the tensor cores' block-scaled MMA (the MXFP8 form of the recipe;
+--no-variant skips it).
+
 --sweep: the micro-batch knee sweep of a 28-layer step (M = 4096 ... 32768 tokens,
 one stream), one JSON line per M and one naming the knee.
 
@@ -168,29 +172,38 @@ class ClockSampler:
 class LayerWork:
     """Device buffers of one step and the launch sequence through the C ABI."""
 
-    def __init__(self, dev, host_inputs, separate=False):
+    def __init__(self, dev, host_inputs, separate=False, scales="fp32"):
         import torch
         import blockwise_fp8_linear_b200 as fb
         self.fb = fb
         self.torch = torch
         self.separate = separate
+        # scales: "fp32" (amax/448, promoted per block on the CUDA cores) or "e8m0" (power
+        # of two, scale blocks applied by the block-scaled MMA)
+        self.e8 = scales == "e8m0"
         self.launches_per_step = (8 if separate else 6) * len(LINEARS)
         self.lin = []
         for (name, din, dout), (X, W, dY) in zip(LINEARS, host_inputs):
             t = lambda a: torch.from_numpy(a.view(np.int16)).view(torch.bfloat16)
+            if self.e8:  # scale blocks of 512 bytes per 128 rows x 128-deep block
+                sc = lambda rows, red: torch.empty(rows // 128, (red // 128) * 512, dtype=torch.uint8,
+                                                   device=dev)
+                scales_ = {"sx": sc(TOKENS, din), "sw": sc(dout, din), "sdy": sc(TOKENS, dout),
+                           "sdyt": sc(dout, TOKENS), "sxt": sc(din, TOKENS)}
+            else:
+                f32 = lambda r, c: torch.empty(r, c, dtype=torch.float32, device=dev)
+                scales_ = {"sx": f32(din // 128, TOKENS), "sw": f32(dout // 128, din // 128),
+                           "sdy": f32(dout // 128, TOKENS), "sdyt": f32(TOKENS // 128, dout),
+                           "sxt": f32(TOKENS // 128, din)}
             d = {
                 "name": name, "din": din, "dout": dout,
                 "X": t(X).to(dev), "W": t(W).to(dev), "dY": t(dY).to(dev),
                 "qx": torch.empty(TOKENS, din, dtype=torch.uint8, device=dev),
-                "sx": torch.empty(din // 128, TOKENS, dtype=torch.float32, device=dev),
                 "qw": torch.empty(dout, din, dtype=torch.uint8, device=dev),
-                "sw": torch.empty(dout // 128, din // 128, dtype=torch.float32, device=dev),
                 "qdy": torch.empty(TOKENS, dout, dtype=torch.uint8, device=dev),
-                "sdy": torch.empty(dout // 128, TOKENS, dtype=torch.float32, device=dev),
                 "qdyt": torch.empty(dout, TOKENS, dtype=torch.uint8, device=dev),
-                "sdyt": torch.empty(TOKENS // 128, dout, dtype=torch.float32, device=dev),
                 "qxt": torch.empty(din, TOKENS, dtype=torch.uint8, device=dev),
-                "sxt": torch.empty(TOKENS // 128, din, dtype=torch.float32, device=dev),
+                **scales_,
                 "Y": torch.empty(TOKENS, dout, dtype=torch.bfloat16, device=dev),
                 "dX": torch.empty(TOKENS, din, dtype=torch.bfloat16, device=dev),
                 "dW": torch.empty(dout, din, dtype=torch.bfloat16, device=dev),
@@ -216,8 +229,9 @@ class LayerWork:
                 e0 = torch.cuda.Event(enable_timing=True)
                 e1 = torch.cuda.Event(enable_timing=True)
                 e0.record(s)
-            rc = L.fp8_gemm_blockwise(mode, a.data_ptr(), sa.data_ptr(), b.data_ptr(),
-                                      sb.data_ptr(), out.data_ptr(), M, N, K, s.cuda_stream)
+            fn = L.fp8_gemm_blockwise_e8m0 if self.e8 else L.fp8_gemm_blockwise
+            rc = fn(mode, a.data_ptr(), sa.data_ptr(), b.data_ptr(), sb.data_ptr(), out.data_ptr(),
+                    M, N, K, s.cuda_stream)
             if rc:
                 raise fb.Fp8bwError(rc, "fp8_gemm_blockwise")
             if gemm_events is not None:
@@ -225,6 +239,11 @@ class LayerWork:
                 gemm_events.append((e0, e1, 2 * M * N * K))
 
         st = main.cuda_stream
+        e8 = self.e8
+        q_act = L.fp8_quant_act_e8m0 if e8 else L.fp8_quant_act
+        q_act_t = L.fp8_quant_act_t_e8m0 if e8 else L.fp8_quant_act_t
+        q_dual = L.fp8_quant_act_dual_e8m0 if e8 else L.fp8_quant_act_dual
+        q_weight = L.fp8_quant_weight_e8m0 if e8 else L.fp8_quant_weight
 
         def chk(rc, what):
             if rc:
@@ -233,21 +252,21 @@ class LayerWork:
         for d in self.lin:
             din, dout = d["din"], d["dout"]
             if self.separate:
-                chk(L.fp8_quant_act(d["X"].data_ptr(), T, din, d["qx"].data_ptr(), d["sx"].data_ptr(), st), "qa")
+                chk(q_act(d["X"].data_ptr(), T, din, d["qx"].data_ptr(), d["sx"].data_ptr(), st), "qa")
             else:  # X read once: row-wise copy for fprop, token-wise copy kept for wgrad
-                chk(L.fp8_quant_act_dual(d["X"].data_ptr(), T, din, d["qx"].data_ptr(), d["sx"].data_ptr(),
-                                         d["qxt"].data_ptr(), d["sxt"].data_ptr(), st), "qd")
-            chk(L.fp8_quant_weight(d["W"].data_ptr(), dout, din, d["qw"].data_ptr(),
-                                   d["sw"].data_ptr(), None, st), "qw")
+                chk(q_dual(d["X"].data_ptr(), T, din, d["qx"].data_ptr(), d["sx"].data_ptr(),
+                           d["qxt"].data_ptr(), d["sxt"].data_ptr(), st), "qd")
+            chk(q_weight(d["W"].data_ptr(), dout, din, d["qw"].data_ptr(),
+                         d["sw"].data_ptr(), None, st), "qw")
             gemm(fb.FPROP, d["qx"], d["sx"], d["qw"], d["sw"], d["Y"], T, dout, din)
             if self.separate:
-                chk(L.fp8_quant_act(d["dY"].data_ptr(), T, dout, d["qdy"].data_ptr(), d["sdy"].data_ptr(), st), "qa")
+                chk(q_act(d["dY"].data_ptr(), T, dout, d["qdy"].data_ptr(), d["sdy"].data_ptr(), st), "qa")
             else:
-                chk(L.fp8_quant_act_dual(d["dY"].data_ptr(), T, dout, d["qdy"].data_ptr(), d["sdy"].data_ptr(),
-                                         d["qdyt"].data_ptr(), d["sdyt"].data_ptr(), st), "qd")
+                chk(q_dual(d["dY"].data_ptr(), T, dout, d["qdy"].data_ptr(), d["sdy"].data_ptr(),
+                           d["qdyt"].data_ptr(), d["sdyt"].data_ptr(), st), "qd")
             if self.separate:
-                chk(L.fp8_quant_act_t(d["dY"].data_ptr(), T, dout, d["qdyt"].data_ptr(), d["sdyt"].data_ptr(), st), "qt")
-                chk(L.fp8_quant_act_t(d["X"].data_ptr(), T, din, d["qxt"].data_ptr(), d["sxt"].data_ptr(), st), "qt")
+                chk(q_act_t(d["dY"].data_ptr(), T, dout, d["qdyt"].data_ptr(), d["sdyt"].data_ptr(), st), "qt")
+                chk(q_act_t(d["X"].data_ptr(), T, din, d["qxt"].data_ptr(), d["sxt"].data_ptr(), st), "qt")
             if side is not None:
                 ready = torch.cuda.Event()
                 ready.record(main)
@@ -405,6 +424,39 @@ def run_ours(args):
         "measured_on": "a separate pass of the same steps on one stream (no kernel overlap)",
     }
 
+    # the same step with power-of-two (E8M0) scales applied by the block-scaled MMA
+    # (the MXFP8 form of the recipe), for comparison; not the headline
+    variant = None
+    if not args.no_variant:
+        work8 = LayerWork(dev, host, separate=args.separate_quant, scales="e8m0")
+        for _ in range(args.warmup):
+            work8.step(side=side)
+        torch.cuda.synchronize()
+        ev8 = []
+        for _ in range(args.steps):
+            work8.step(ev8)
+        v0 = torch.cuda.Event(enable_timing=True)
+        v1 = torch.cuda.Event(enable_timing=True)
+        barrier(world)
+        torch.cuda.synchronize()
+        v0.record()
+        for _ in range(args.steps):
+            work8.step(side=side)
+        v1.record()
+        torch.cuda.synchronize()
+        barrier(world)
+        if fb.fp8bw_last_device_error() != 0:
+            raise RuntimeError("a bounded in-kernel wait ran out in the E8M0 variant")
+        v_ms = max_over_ranks(v0.elapsed_time(v1), world) / args.steps
+        g8_ms = sum(e0.elapsed_time(e1) for e0, e1, _ in ev8)
+        g8 = sum(f for _, _, f in ev8) / (g8_ms * 1e-3) / 1e12
+        variant = {"scales": "e8m0 (power of two, scale blocks applied by tcgen05.mma block_scale)",
+                   "value": round(world * STEP_FLOPS / (v_ms * 1e-3) / 1e12, 3), "unit": UNIT,
+                   "ms_per_step": round(v_ms, 4), "gemm_tflops": round(g8, 2),
+                   "gemm_frac": round(g8 / (measured_peaks()[0]["bf16_tflops"] * FP8_OVER_BF16), 4),
+                   "gemm_kernel": "fp8_gemm_mx_kernel"}
+        del work8
+
     cpu = None
     if rank == 0 and not args.no_cpu:
         cpu = cpu_baseline(budget_s=args.cpu_budget, host=host)
@@ -420,6 +472,7 @@ def run_ours(args):
             "e2e": e2e, "gpu_launches": work.launches_per_step * args.steps,
             "clocks": clock_info,
             "pct_of_fp8_peak": round(100 * value / world / fp8_peak, 2),
+            "variant_e8m0": variant,
         }
         print(json.dumps(line), flush=True)
     if world > 1:
@@ -508,7 +561,8 @@ def run_reference(args):
     print(json.dumps(line), flush=True)
 
 
-KERNEL_CASES = ("gemm_fprop", "gemm_dgrad", "gemm_wgrad", "quant_act", "quant_act_t",
+KERNEL_CASES = ("gemm_fprop", "gemm_dgrad", "gemm_wgrad", "gemm_mx_fprop", "gemm_mx_wgrad",
+                "quant_dual_e8m0", "quant_act", "quant_act_t",
                 "quant_dual", "quant_weight")
 
 
@@ -528,7 +582,18 @@ def run_kernel_only(args):
     def randn(r, c, std):
         return (torch.randn(r, c, device=dev, generator=g) * std).to(torch.bfloat16)
 
-    if case.startswith("gemm"):
+    if case.startswith("gemm_mx"):
+        X, W, dY = randn(T, din, 1.0), randn(dout, din, 0.02), randn(T, dout, 1e-3)
+        if case == "gemm_mx_fprop":
+            a, sa = fb.fp8_quant_act_e8m0(X)
+            b, sb, _ = fb.fp8_quant_weight_e8m0(W)
+            launch = lambda: fb.fp8_gemm_blockwise_e8m0(fb.FPROP, a, sa, b, sb, T, dout, din)
+        else:
+            a, sa = fb.fp8_quant_act_t_e8m0(dY)
+            b, sb = fb.fp8_quant_act_t_e8m0(X)
+            launch = lambda: fb.fp8_gemm_blockwise_e8m0(fb.WGRAD, a, sa, b, sb, dout, din, T)
+        work = ("TFLOP/s", 2 * T * din * dout / 1e12)
+    elif case.startswith("gemm"):
         X, W, dY = randn(T, din, 1.0), randn(dout, din, 0.02), randn(T, dout, 1e-3)
         qw, sw, _ = fb.fp8_quant_weight(W)
         if case == "gemm_fprop":
@@ -554,9 +619,11 @@ def run_kernel_only(args):
             launch = lambda: fb.fp8_quant_act_t(X)
         elif case == "quant_dual":
             launch = lambda: fb.fp8_quant_act_dual(X)
+        elif case == "quant_dual_e8m0":
+            launch = lambda: fb.fp8_quant_act_dual_e8m0(X)
         else:
             launch = lambda: fb.fp8_quant_weight(X)
-        per_elem = (4 + 8 / 128) if case == "quant_dual" else (3 + 4 / 128)
+        per_elem = (4 + 8 / 128) if case.startswith("quant_dual") else (3 + 4 / 128)
         work = ("GB/s", R * C * per_elem / 1e9)
     torch.cuda.synchronize()
     for _ in range(args.warmup):
@@ -699,6 +766,8 @@ def main():
     ap.add_argument("--separate-quant", action="store_true",
                     help="quantize X and dY with separate row-wise and token-wise passes "
                          "instead of the fused dual-output quantizer")
+    ap.add_argument("--no-variant", action="store_true",
+                    help="skip the power-of-two (E8M0) scale variant of the step")
     ap.add_argument("--no-overlap", action="store_true",
                     help="run every kernel on one stream (no dgrad/wgrad overlap)")
     ap.add_argument("--kernel-only", choices=KERNEL_CASES, default=None,
