@@ -212,12 +212,14 @@ class LayerWork:
         self.h2d_bytes = sum(d[k].numel() * 2 for d in self.lin for k in ("X", "W", "dY"))
         self.d2h_bytes = sum(d[k].numel() * 2 for d in self.lin for k in ("Y", "dX", "dW"))
 
-    def step(self, gemm_events=None, side=None):
+    def step(self, gemm_events=None, side=None, hooks=None):
         """Enqueue one step on the current stream.  gemm_events: optional list that
         receives (start, end, flops) CUDA-event triples around each GEMM.  side: an
         optional second stream; each linear's wgrad then runs there, after the dY
         quantizer and concurrently with the dgrad (the two are independent given
-        dY), and the current stream waits for it at the end of the step."""
+        dY), and the current stream waits for it at the end of the step.
+        hooks: optional object with before(i), inputs_read(i) and after(i, main, side)
+        called around linear i (used by the end-to-end pipeline)."""
         fb, torch = self.fb, self.torch
         L = fb.lib()
         main = torch.cuda.current_stream()
@@ -249,8 +251,10 @@ class LayerWork:
             if rc:
                 raise fb.Fp8bwError(rc, what)
 
-        for d in self.lin:
+        for i, d in enumerate(self.lin):
             din, dout = d["din"], d["dout"]
+            if hooks is not None:
+                hooks.before(i)
             if self.separate:
                 chk(q_act(d["X"].data_ptr(), T, din, d["qx"].data_ptr(), d["sx"].data_ptr(), st), "qa")
             else:  # X read once: row-wise copy for fprop, token-wise copy kept for wgrad
@@ -267,12 +271,16 @@ class LayerWork:
             if self.separate:
                 chk(q_act_t(d["dY"].data_ptr(), T, dout, d["qdyt"].data_ptr(), d["sdyt"].data_ptr(), st), "qt")
                 chk(q_act_t(d["X"].data_ptr(), T, din, d["qxt"].data_ptr(), d["sxt"].data_ptr(), st), "qt")
+            if hooks is not None:
+                hooks.inputs_read(i)
             if side is not None:
                 ready = torch.cuda.Event()
                 ready.record(main)
                 side.wait_event(ready)
             gemm(fb.DGRAD, d["qdy"], d["sdy"], d["qw"], d["sw"], d["dX"], T, din, dout)
             gemm(fb.WGRAD, d["qdyt"], d["sdyt"], d["qxt"], d["sxt"], d["dW"], dout, din, T, stream=side)
+            if hooks is not None:
+                hooks.after(i, main, side if side is not None else main)
         if side is not None:
             done = torch.cuda.Event()
             done.record(side)
@@ -382,16 +390,53 @@ def run_ours(args):
                     torch.empty(d["dX"].shape, dtype=torch.int16).pin_memory(),
                     torch.empty(d["dW"].shape, dtype=torch.int16).pin_memory()) for d in work.lin]
 
+        # Pipelined per linear over three streams: uploads (h2d), compute (the current
+        # stream, wgrad on `side`), downloads (d2h).  Events order every buffer's
+        # writer after its previous reader: an upload after the previous step's
+        # quantizers of that linear, the compute after its upload and after the
+        # previous step's download of its outputs, a download after the compute.
+        h2d, d2h = torch.cuda.Stream(device=dev), torch.cuda.Stream(device=dev)
+        n_lin = len(work.lin)
+        mk = lambda: [torch.cuda.Event() for _ in range(n_lin)]
+        ev = {"in_free": mk(), "up": mk(), "done_main": mk(), "done_side": mk(), "out_read": mk()}
+        for k in ("in_free", "done_side", "out_read"):
+            for e in ev[k]:
+                e.record()
+
+        class Hooks:
+            def before(self, i):
+                main = torch.cuda.current_stream()
+                main.wait_event(ev["up"][i])
+                main.wait_event(ev["out_read"][i])
+                main.wait_event(ev["done_side"][i])
+
+            def inputs_read(self, i):
+                ev["in_free"][i].record()
+
+            def after(self, i, main, side_s):
+                ev["done_main"][i].record(main)
+                ev["done_side"][i].record(side_s)
+                d = work.lin[i]
+                Y, dX, dW = pin_out[i]
+                d2h.wait_event(ev["done_main"][i])
+                d2h.wait_event(ev["done_side"][i])
+                with torch.cuda.stream(d2h):
+                    Y.copy_(d["Y"].view(torch.int16), non_blocking=True)
+                    dX.copy_(d["dX"].view(torch.int16), non_blocking=True)
+                    dW.copy_(d["dW"].view(torch.int16), non_blocking=True)
+                ev["out_read"][i].record(d2h)
+
+        hooks = Hooks()
+
         def e2e_step():
-            for d, (X, W, dY) in zip(work.lin, pin_in):
-                d["X"].view(torch.int16).copy_(X, non_blocking=True)
-                d["W"].view(torch.int16).copy_(W, non_blocking=True)
-                d["dY"].view(torch.int16).copy_(dY, non_blocking=True)
-            work.step(side=side)
-            for d, (Y, dX, dW) in zip(work.lin, pin_out):
-                Y.copy_(d["Y"].view(torch.int16), non_blocking=True)
-                dX.copy_(d["dX"].view(torch.int16), non_blocking=True)
-                dW.copy_(d["dW"].view(torch.int16), non_blocking=True)
+            for i, (d, (X, W, dY)) in enumerate(zip(work.lin, pin_in)):
+                h2d.wait_event(ev["in_free"][i])
+                with torch.cuda.stream(h2d):
+                    d["X"].view(torch.int16).copy_(X, non_blocking=True)
+                    d["W"].view(torch.int16).copy_(W, non_blocking=True)
+                    d["dY"].view(torch.int16).copy_(dY, non_blocking=True)
+                ev["up"][i].record(h2d)
+            work.step(side=side, hooks=hooks)
 
         e2e_step()
         torch.cuda.synchronize()
@@ -402,6 +447,7 @@ def run_ours(args):
         a0.record()
         for _ in range(n_e2e):
             e2e_step()
+        torch.cuda.current_stream().wait_stream(d2h)
         a1.record()
         torch.cuda.synchronize()
         barrier(world)
