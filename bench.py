@@ -55,7 +55,7 @@ STEP_FLOPS = sum(3 * 2 * TOKENS * din * dout for _, din, dout in LINEARS)
 FP8_OVER_BF16 = 4.5 / 2.25  # nominal dense FP8 : BF16 tensor throughput on B200
 
 
-def config_dict(n, overlap=True):
+def config_dict(n, overlap=True, dp_grad=False):
     return {
         "schedule": ("each linear's wgrad on a second stream, concurrent with its dgrad"
                      if overlap else "one stream"),
@@ -65,7 +65,8 @@ def config_dict(n, overlap=True):
         "passes": "fprop+dgrad+wgrad with all quantizers (X and dY quantized once into both layouts)",
         "step_gflop": round(STEP_FLOPS / 1e9, 3),
         "l2": "inputs larger than L2 (637 MB of BF16 inputs per step), no flush",
-        "parallelism": f"replicas x{n}" if n > 1 else "single GPU",
+        "parallelism": (f"dp{n}, dW reduce-scatter (NCCL) overlapped with the next linear" if dp_grad
+                        else f"replicas x{n}" if n > 1 else "single GPU"),
     }
 
 
@@ -212,7 +213,7 @@ class LayerWork:
         self.h2d_bytes = sum(d[k].numel() * 2 for d in self.lin for k in ("X", "W", "dY"))
         self.d2h_bytes = sum(d[k].numel() * 2 for d in self.lin for k in ("Y", "dX", "dW"))
 
-    def step(self, gemm_events=None, side=None, hooks=None):
+    def step(self, gemm_events=None, side=None, hooks=None, reducer=None):
         """Enqueue one step on the current stream.  gemm_events: optional list that
         receives (start, end, flops) CUDA-event triples around each GEMM.  side: an
         optional second stream; each linear's wgrad then runs there, after the dY
@@ -279,12 +280,16 @@ class LayerWork:
                 side.wait_event(ready)
             gemm(fb.DGRAD, d["qdy"], d["sdy"], d["qw"], d["sw"], d["dX"], T, din, dout)
             gemm(fb.WGRAD, d["qdyt"], d["sdyt"], d["qxt"], d["sxt"], d["dW"], dout, din, T, stream=side)
+            if reducer is not None:
+                reducer.launch(i, d["dW"], side if side is not None else main)
             if hooks is not None:
                 hooks.after(i, main, side if side is not None else main)
         if side is not None:
             done = torch.cuda.Event()
             done.record(side)
             main.wait_event(done)
+        if reducer is not None:
+            reducer.wait()
 
 
 def make_inputs(rank=0):
@@ -297,6 +302,41 @@ def make_inputs(rank=0):
         dY = synth.normal_bf16(TOKENS, dout, 1e-3, seed=synth.seed_for(wl, 2 + 10 * rank))
         out.append((X, W, dY))
     return out
+
+
+class DpGradReducer:
+    """Data-parallel weight-gradient exchange: each linear's dW [out][in] is summed over
+    the ranks and split by rows, rank r keeping rows [r*out/N, (r+1)*out/N) (a
+    reduce-scatter, the gradient layout of an optimizer sharded by rows).  On GPUs the
+    collective is NCCL over NVLink, issued on the stream that computed dW so that it
+    overlaps the next linear's kernels; wait() makes the current stream wait for all
+    of them.  CPU tensors and the gloo backend take the same path (for tests)."""
+
+    def __init__(self, shapes, world, device):
+        import torch
+        self.world = world
+        self.shards = [torch.empty(dout // world, din, dtype=torch.bfloat16, device=device)
+                       for dout, din in shapes]
+        self.pending = []
+
+    @staticmethod
+    def rows(dout, world, rank):
+        return rank * dout // world, (rank + 1) * dout // world
+
+    def launch(self, i, dW, stream=None):
+        import torch
+        import torch.distributed as dist
+        if stream is not None:
+            with torch.cuda.stream(stream):
+                h = dist.reduce_scatter_tensor(self.shards[i], dW, op=dist.ReduceOp.SUM, async_op=True)
+        else:
+            h = dist.reduce_scatter_tensor(self.shards[i], dW, op=dist.ReduceOp.SUM, async_op=True)
+        self.pending.append(h)
+
+    def wait(self):
+        for h in self.pending:
+            h.wait()
+        self.pending.clear()
 
 
 def barrier(world):
@@ -334,10 +374,13 @@ def run_ours(args):
     host = make_inputs(rank)
     work = LayerWork(dev, host, separate=args.separate_quant)
     side = None if args.no_overlap else torch.cuda.Stream(device=dev)
+    reducer = None
+    if world > 1 and args.dp_grad == "reduce-scatter":
+        reducer = DpGradReducer([(dout, din) for _, din, dout in LINEARS], world, dev)
 
     # warm-up
     for _ in range(args.warmup):
-        work.step(side=side)
+        work.step(side=side, reducer=reducer)
     torch.cuda.synchronize()
     if fb.fp8bw_last_device_error() != 0:
         raise RuntimeError("a bounded in-kernel wait ran out during warm-up")
@@ -366,7 +409,7 @@ def run_ours(args):
         t1 = torch.cuda.Event(enable_timing=True)
         t0.record()
         for _ in range(args.steps):
-            work.step(side=side)
+            work.step(side=side, reducer=reducer)
         t1.record()
         torch.cuda.synchronize()
         barrier(world)
@@ -513,7 +556,8 @@ def run_ours(args):
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_per_step, 4),
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
             "dtype": "e4m3", "data": "synthetic (seeded splitmix64/Box-Muller BF16)",
-            "config": config_dict(world, overlap=side is not None), "roofline": roofline,
+            "config": config_dict(world, overlap=side is not None,
+                                  dp_grad=reducer is not None), "roofline": roofline,
             "cpu_baseline": cpu,
             "e2e": e2e, "gpu_launches": work.launches_per_step * args.steps,
             "clocks": clock_info,
@@ -812,6 +856,9 @@ def main():
     ap.add_argument("--separate-quant", action="store_true",
                     help="quantize X and dY with separate row-wise and token-wise passes "
                          "instead of the fused dual-output quantizer")
+    ap.add_argument("--dp-grad", choices=["none", "reduce-scatter"], default="none",
+                    help="with N > 1: none = independent replicas; reduce-scatter = sum each "
+                         "linear's dW over the ranks (NCCL), overlapped with the next linear")
     ap.add_argument("--no-variant", action="store_true",
                     help="skip the power-of-two (E8M0) scale variant of the step")
     ap.add_argument("--no-overlap", action="store_true",
