@@ -189,3 +189,13 @@ def test_gemm_e8m0_zero_and_deterministic(mode):
     y1 = fp8_gemm_blockwise_e8m0(mode, a, sa, b, sb, M, N, K)
     y2 = fp8_gemm_blockwise_e8m0(mode, a, sa, b, sb, M, N, K)
     assert torch.equal(y1.view(torch.int16), y2.view(torch.int16))
+
+
+@pytest.mark.parametrize("mode", [FPROP, DGRAD, WGRAD])
+def test_gemm_e8m0_sweep_size_sampled(mode):
+    """The largest micro-batch of the sweep (M = 32768 tokens): the wgrad reduction runs
+    over 256 blocks of 128 tokens in one accumulator."""
+    T, Din, Dout = 32768, 6144, 2048
+    X, W, dY = _layer(T, Din, Dout, seed=90 + mode)
+    y, y_ref, asum = _run(mode, X, W, dY, sample=8)
+    check_gemm(y, y_ref, asum, f"e8m0 down M=32768 mode {mode}")
