@@ -18,14 +18,16 @@
 //               blocks of 128 rows: row r's code at bytes 16 (r % 32) + 4 (r / 32),
 //               repeated four times for the four 32-wide K steps), so scale factors
 //               travel by TMA with the operands and need no rewriting on chip.
-//   warp 1      MMA issuer (even CTA): per block, tcgen05.cp of the stage's scale
-//               blocks into tensor memory, then four block-scaled MMAs into the
-//               tile's accumulator.
+//   warp 1      MMA issuer (even CTA): per block, four block-scaled MMAs into the
+//               tile's accumulator, reading the stage's scale factors from tensor memory.
+//   warp 2      scale copier (even CTA): per block, tcgen05.cp of the stage's scale
+//               blocks into that stage's tensor-memory region, so the MMA issuer's
+//               thread issues nothing but MMAs and commits.
 //   warps 4-11  epilogue: after the tile's last block, load the accumulator from TMEM,
 //               release it to the MMA issuer, round to BF16 and store through swizzled
 //               shared memory with TMA.
-// Tensor memory: the accumulator (BN columns), then 4 columns of A scale factors and
-// 4 per 128 columns of B scale factors.
+// Tensor memory: the accumulator (BN columns), then one 16-column region per pipeline
+// stage holding 4 columns of A scale factors and 4 per 128 columns of B scale factors.
 //
 // Every wait is bounded (about one second); a wait that runs out records an error
 // code and the CTA (pair) unwinds.
@@ -75,11 +77,12 @@ struct MxCfg {
     static constexpr int BAR_OFF = OUT_OFF + EPI_WARPS * OUT_WARP;
     static constexpr int SMEM = 1024 + BAR_OFF + 256;
     static constexpr int TMEM_COLS = 512;
-    static constexpr int SFA_COL = BN;
-    static constexpr int SFB_COL = BN + 4;
+    static constexpr int SF_COL = BN;                      // first scale-factor region
+    static constexpr int SF_COLS = 16;                     // per stage: A (4), then B (4 each)
     static_assert(COLS % 64 == 0, "epilogue works in 64-column boxes");
     static_assert(B_ROWS % B_BOX == 0, "B rows must be whole boxes");
-    static_assert(SFB_COL + 4 * NSFB <= TMEM_COLS, "tensor memory budget");
+    static_assert(4 * (1 + NSFB) <= SF_COLS, "scale factors of one stage");
+    static_assert(SF_COL + STAGES * SF_COLS <= TMEM_COLS, "tensor memory budget");
     static_assert(SMEM <= 227 * 1024, "shared memory budget");
 };
 
@@ -116,7 +119,8 @@ fp8_gemm_mx_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constan
     uint64_t *empty = full + STAGES;       // [STAGES] MMA -> TMA
     uint64_t *tfull = empty + STAGES;      // MMA -> epilogue
     uint64_t *tempty = tfull + 1;          // epilogue -> MMA (even CTA)
-    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(tempty + 1);
+    uint64_t *sfr = tempty + 1;            // [STAGES] scale copier -> MMA (even CTA)
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(sfr + STAGES);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -132,6 +136,7 @@ fp8_gemm_mx_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constan
         for (int s = 0; s < STAGES; ++s) {
             mbar_init(&full[s], 1);
             mbar_init(&empty[s], 1);
+            mbar_init(&sfr[s], 1);
         }
         mbar_init(tfull, 1);
         mbar_init(tempty, EPI_WARPS * CG);
@@ -226,26 +231,25 @@ fp8_gemm_mx_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constan
             int stage = 0;
             uint32_t phase = 0;
             const uint32_t d_tmem = tmem_base;
-            const uint32_t sfa_tmem = tmem_base + Cfg::SFA_COL;
-            const uint32_t sfb_tmem = tmem_base + Cfg::SFB_COL;
             for (int i = 0; i < my_tiles && !*abort_flag; ++i) {
                 // the epilogue has drained the accumulator of the previous tile
                 if (!mbar_wait_bounded(tempty, uint32_t(i & 1) ^ 1u, abort_flag, &g_mx_error,
                                        MXE_TEMPTY, MX_WAIT_NS))
                     goto role_done;
                 for (int kb = 0; kb < KB; ++kb) {
-                    if (!mbar_spin_bounded(&full[stage], phase, abort_flag, &g_mx_error, MXE_MMA,
+                    // the stage's scale factors are in tensor memory (which implies its
+                    // operands have landed); the full barrier is tested for the operands'
+                    // own visibility and has completed by then
+                    if (!mbar_spin_bounded(&sfr[stage], phase, abort_flag, &g_mx_error, MXE_MMA,
+                                           MX_WAIT_NS) ||
+                        !mbar_spin_bounded(&full[stage], phase, abort_flag, &g_mx_error, MXE_MMA,
                                            MX_WAIT_NS))
                         goto role_done;
                     tc_fence_after();
                     const uint32_t a_addr = smem_u32(smem + stage * Cfg::STAGE_BYTES);
                     const uint32_t b_addr = a_addr + Cfg::A_BYTES;
-                    const uint32_t sf_addr = b_addr + Cfg::B_BYTES;
-                    tmem_cp_32x128b_warpx4<CG>(sfa_tmem, make_smem_desc_rows16(sf_addr));
-#pragma unroll
-                    for (int q = 0; q < Cfg::NSFB; ++q)
-                        tmem_cp_32x128b_warpx4<CG>(sfb_tmem + 4 * q,
-                                                   make_smem_desc_rows16(sf_addr + 512 * (1 + q)));
+                    const uint32_t sfa_tmem = tmem_base + uint32_t(Cfg::SF_COL + stage * Cfg::SF_COLS);
+                    const uint32_t sfb_tmem = sfa_tmem + 4;
 #pragma unroll
                     for (int k = 0; k < MX_BK / 32; ++k) {
                         const uint64_t adesc = make_smem_desc_sw128(a_addr + k * 32, 16, 1024);
@@ -271,6 +275,37 @@ fp8_gemm_mx_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constan
                     mma_commit(tfull);
                 else
                     mma_commit_pair(tfull, 0x3);
+            }
+        } else if (warp == 2 && lane == 0 && rank == 0) {
+            // ---------------------------------------------------------- scale copier
+            // Per stage: tcgen05.cp of its scale blocks into the stage's own tensor-memory
+            // region, signalled to the MMA issuer by a commit.  A region is rewritten only
+            // after the producer has seen the stage's MMAs complete (empty) and refilled it
+            // (full), so the copy never overtakes the MMAs that read the previous contents.
+            int stage = 0;
+            uint32_t phase = 0;
+            const int blocks = my_tiles * KB;
+            for (int j = 0; j < blocks && !*abort_flag; ++j) {
+                if (!mbar_spin_bounded(&full[stage], phase, abort_flag, &g_mx_error, MXE_MMA,
+                                       MX_WAIT_NS))
+                    goto role_done;
+                tc_fence_after();
+                const uint32_t sf_addr =
+                    smem_u32(smem + stage * Cfg::STAGE_BYTES) + Cfg::A_BYTES + Cfg::B_BYTES;
+                const uint32_t sfa_tmem = tmem_base + uint32_t(Cfg::SF_COL + stage * Cfg::SF_COLS);
+                tmem_cp_32x128b_warpx4<CG>(sfa_tmem, make_smem_desc_rows16(sf_addr));
+#pragma unroll
+                for (int q = 0; q < Cfg::NSFB; ++q)
+                    tmem_cp_32x128b_warpx4<CG>(sfa_tmem + 4 + 4 * q,
+                                               make_smem_desc_rows16(sf_addr + 512 * (1 + q)));
+                if (CG == 1)
+                    mma_commit(&sfr[stage]);
+                else
+                    mma_commit_pair(&sfr[stage], 0x1);
+                if (++stage == STAGES) {
+                    stage = 0;
+                    phase ^= 1u;
+                }
             }
         }
     role_done:;
