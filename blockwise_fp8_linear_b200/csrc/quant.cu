@@ -49,14 +49,18 @@ struct GroupDiv {
 __device__ __forceinline__ float bf16lo(uint32_t w) { return __uint_as_float(w << 16); }
 __device__ __forceinline__ float bf16hi(uint32_t w) { return __uint_as_float(w & 0xFFFF0000u); }
 
-// Fast-path quotients of a pair of values by per-lane-half scales (s, r, -s given as
-// packed pairs): q0 = x*r, e = x - q0*s (one FMA, exact), q = q0 + e*r.
-__device__ __forceinline__ float2 div2_fast(float2 x, float2 r, float2 neg_s)
+// Fast-path quotients of a pair of values by per-lane-half scales (r, -r and s given
+// as packed pairs): q0 = x*r, d = q0*s - x (one FMA, exact), q = q0 - d*r.  The
+// residual is taken as q0*s - x rather than x - q0*s so that zeros keep their sign
+// with no fix-up: for x = +-0, q0 = +-0 and d = +0, so q = (-0) + (+-0) = +-0; when
+// q0 underflows to a zero, d = -x exactly and q = x*r + q0 carries the sign of x; and
+// q0 - d*r cannot cancel exactly to zero for a nonzero q0, because |d*r| is within
+// an ulp of |q0 - x/s|, far below |q0|.
+__device__ __forceinline__ float2 div2_fast(float2 x, float2 r, float2 neg_r, float2 s)
 {
     const float2 q0 = __fmul2_rn(x, r);
-    const float2 e = __ffma2_rn(q0, neg_s, x);
-    const float2 q = __ffma2_rn(e, r, q0);
-    return make_float2(copysignf(q.x, x.x), copysignf(q.y, x.y));
+    const float2 d = __ffma2_rn(q0, s, make_float2(-x.x, -x.y));
+    return __ffma2_rn(d, neg_r, q0);
 }
 
 // |bf16| max over two packed words, as packed unsigned 16-bit halves (for
@@ -72,24 +76,34 @@ __device__ __forceinline__ float halves_max_to_float(uint32_t m2)
     return __uint_as_float(m << 16);
 }
 
-// Eight BF16 values of one group (one uint4) -> eight E4M3 codes (one uint2).
-__device__ __forceinline__ uint2 quant8(uint4 v, const GroupDiv &d)
+// Eight BF16 values of one group (one uint4) -> eight E4M3 codes (one uint2), by the
+// fast path (r = RN(1/s)) or by IEEE division.
+__device__ __forceinline__ uint2 quant8_fast(uint4 v, float r, float s)
+{
+    const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+    const float2 r2 = make_float2(r, r), nr2 = make_float2(-r, -r), s2 = make_float2(s, s);
+    uint32_t c[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        const float2 q = div2_fast(make_float2(bf16lo(w[i]), bf16hi(w[i])), r2, nr2, s2);
+        c[i] = cvt_e4m3x2(q.x, q.y);
+    }
+    return make_uint2(c[0] | (c[1] << 16), c[2] | (c[3] << 16));
+}
+
+__device__ __forceinline__ uint2 quant8_ieee(uint4 v, float s)
 {
     const uint32_t w[4] = {v.x, v.y, v.z, v.w};
     uint32_t c[4];
-    if (d.fast) {
-        const float2 r2 = make_float2(d.r, d.r), ns2 = make_float2(-d.s, -d.s);
 #pragma unroll
-        for (int i = 0; i < 4; ++i) {
-            const float2 q = div2_fast(make_float2(bf16lo(w[i]), bf16hi(w[i])), r2, ns2);
-            c[i] = cvt_e4m3x2(q.x, q.y);
-        }
-    } else {
-#pragma unroll
-        for (int i = 0; i < 4; ++i)
-            c[i] = cvt_e4m3x2(__fdiv_rn(bf16lo(w[i]), d.s), __fdiv_rn(bf16hi(w[i]), d.s));
-    }
+    for (int i = 0; i < 4; ++i)
+        c[i] = cvt_e4m3x2(__fdiv_rn(bf16lo(w[i]), s), __fdiv_rn(bf16hi(w[i]), s));
     return make_uint2(c[0] | (c[1] << 16), c[2] | (c[3] << 16));
+}
+
+__device__ __forceinline__ uint2 quant8(uint4 v, const GroupDiv &d)
+{
+    return d.fast ? quant8_fast(v, d.r, d.s) : quant8_ieee(v, d.s);
 }
 
 // Power-of-two (E8M0) scales, the MXFP8 form of the recipe (same section): the group
@@ -244,11 +258,12 @@ quant_act_t_kernel(const uint32_t *__restrict__ x, int64_t M, int64_t K,
     uint32_t clo[4] = {0u, 0u, 0u, 0u}, chi[4] = {0u, 0u, 0u, 0u};
     const GroupDiv dlo(s_lo), dhi(s_hi);
     if (dlo.fast && dhi.fast) {
-        const float2 r2 = make_float2(dlo.r, dhi.r), ns2 = make_float2(-s_lo, -s_hi);
+        const float2 r2 = make_float2(dlo.r, dhi.r), nr2 = make_float2(-dlo.r, -dhi.r);
+        const float2 s2 = make_float2(s_lo, s_hi);
 #pragma unroll
         for (int r = 0; r < 16; r += 2) {
-            const float2 a = div2_fast(make_float2(bf16lo(v[r]), bf16hi(v[r])), r2, ns2);
-            const float2 b = div2_fast(make_float2(bf16lo(v[r + 1]), bf16hi(v[r + 1])), r2, ns2);
+            const float2 a = div2_fast(make_float2(bf16lo(v[r]), bf16hi(v[r])), r2, nr2, s2);
+            const float2 b = div2_fast(make_float2(bf16lo(v[r + 1]), bf16hi(v[r + 1])), r2, nr2, s2);
             clo[r / 4] |= cvt_e4m3x2(a.x, b.x) << (16 * ((r / 2) & 1));
             chi[r / 4] |= cvt_e4m3x2(a.y, b.y) << (16 * ((r / 2) & 1));
         }
@@ -371,8 +386,12 @@ constexpr int QD_THREADS = 256;
 // E8: power-of-two scales in 512-byte blocks (see sf_block_off): s holds
 // [M/128][K/128] blocks (row m of block (m/128, kb)), st holds [K/128][M/128] blocks
 // (column k of X is row k % 128 of block (k/128, mb)).
+// Four CTAs per SM (at most 64 registers): more tiles' loads in flight per SM.
+#ifndef FP8BW_QD_MINB
+#define FP8BW_QD_MINB 4
+#endif
 template <bool ROWS, bool COLS, bool E8 = false>
-__global__ void __launch_bounds__(QD_THREADS)
+__global__ void __launch_bounds__(QD_THREADS, FP8BW_QD_MINB)
 quant_tile_kernel(const uint4 *__restrict__ x, int64_t M, int64_t K, uint2 *__restrict__ q,
                   void *__restrict__ s_out, uint8_t *__restrict__ qt, void *__restrict__ st_out)
 {
@@ -388,36 +407,82 @@ quant_tile_kernel(const uint4 *__restrict__ x, int64_t M, int64_t K, uint2 *__re
         const int64_t m = mb * 128 + p * 16 + rsub;
         v[p] = __ldg(x + (m * K + kb * 128) / 8 + sub);
     }
+    if (ROWS) {
+        // Row groups: half-warp h holds rows 16p + rsub (p < 8), 8 values per lane.
+        // Each lane's partial amax for its 8 rows goes through a transposing reduction
+        // over the 16 lanes (recursive halving: exchange half of the rows' partials with
+        // the lane 8, 4, 2 apart, then combine with the lane 1 apart), after which
+        // lanes 2p and 2p + 1 hold the amax of row 16p + rsub.  Each lane then works out
+        // the scale of that one group, and the quantizing loop fetches group p's
+        // scalars by shuffle: the per-group division and reciprocal run once per lane
+        // for all 8 groups instead of once per group.
+        uint32_t mx[8];
 #pragma unroll
-    for (int p = 0; p < 8; ++p) {
-        const int row = p * 16 + rsub;
-        if (ROWS) {
-            uint32_t m2 = __vmaxu2(absmax2(v[p].x, v[p].y), absmax2(v[p].z, v[p].w));
+        for (int p = 0; p < 8; ++p)
+            mx[p] = __vmaxu2(absmax2(v[p].x, v[p].y), absmax2(v[p].z, v[p].w));
+        {
+            const bool b = (sub & 8) != 0;
 #pragma unroll
-            for (int o = 8; o >= 1; o >>= 1)
-                m2 = __vmaxu2(m2, __shfl_xor_sync(0xffffffffu, m2, o));
-            const float amax = halves_max_to_float(m2);
+            for (int j = 0; j < 4; ++j) {
+                const uint32_t send = b ? mx[j] : mx[j + 4], keep = b ? mx[j + 4] : mx[j];
+                mx[j] = __vmaxu2(keep, __shfl_xor_sync(0xffffffffu, send, 8));
+            }
+        }
+        {
+            const bool b = (sub & 4) != 0;
+#pragma unroll
+            for (int j = 0; j < 2; ++j) {
+                const uint32_t send = b ? mx[j] : mx[j + 2], keep = b ? mx[j + 2] : mx[j];
+                mx[j] = __vmaxu2(keep, __shfl_xor_sync(0xffffffffu, send, 4));
+            }
+        }
+        {
+            const bool b = (sub & 2) != 0;
+            const uint32_t send = b ? mx[0] : mx[1], keep = b ? mx[1] : mx[0];
+            mx[0] = __vmaxu2(keep, __shfl_xor_sync(0xffffffffu, send, 2));
+        }
+        mx[0] = __vmaxu2(mx[0], __shfl_xor_sync(0xffffffffu, mx[0], 1));
+        const float amax = halves_max_to_float(mx[0]);
+        const int64_t m_own = mb * 128 + (sub >> 1) * 16 + rsub;
+        // per group: E8 the multiplier 2^-e (0 for an all-zero group); FP32 the scale
+        // (0 for an all-zero group) and RN(1/s), or -1 when the group takes IEEE division
+        float g0 = 0.0f, g1 = 0.0f;
+        if constexpr (E8) {
+            const int e = e8m0_exponent(amax);
+            g0 = amax != 0.0f ? pow2_neg(e) : 0.0f;
+            if ((sub & 1) == 0)
+                *reinterpret_cast<uint32_t *>(static_cast<uint8_t *>(s_out) +
+                                              ((m_own >> 7) * (K / 128) + kb) * 512 +
+                                              sf_block_off(int(m_own & 127))) = rep4_code(e, amax);
+        } else {
+            g0 = __fdiv_rn(amax, 448.0f);
+            const GroupDiv d(g0);
+            g1 = d.fast ? d.r : -1.0f;
+            if ((sub & 1) == 0)
+                static_cast<float *>(s_out)[kb * M + m_own] = g0;
+        }
+#pragma unroll
+        for (int p = 0; p < 8; ++p) {
+            const int row = p * 16 + rsub;
             const int64_t m = mb * 128 + row;
+            const float gp = __shfl_sync(0xffffffffu, g0, 2 * p, 16);
             uint2 codes = make_uint2(0u, 0u);
             if constexpr (E8) {
-                const int e = e8m0_exponent(amax);
-                if (amax != 0.0f)
-                    codes = quant8_pow2(v[p], pow2_neg(e));
-                if (sub == 0)
-                    *reinterpret_cast<uint32_t *>(static_cast<uint8_t *>(s_out) +
-                                                  ((m >> 7) * (K / 128) + kb) * 512 + sf_block_off(int(m & 127))) =
-                        rep4_code(e, amax);
+                if (gp != 0.0f)
+                    codes = quant8_pow2(v[p], gp);
             } else {
-                const float sc = __fdiv_rn(amax, 448.0f);
-                if (amax != 0.0f)
-                    codes = quant8(v[p], GroupDiv(sc));
-                if (sub == 0)
-                    static_cast<float *>(s_out)[kb * M + m] = sc;
+                const float rp = __shfl_sync(0xffffffffu, g1, 2 * p, 16);
+                if (gp != 0.0f)
+                    codes = rp > 0.0f ? quant8_fast(v[p], rp, gp) : quant8_ieee(v[p], gp);
             }
             q[(m * K + kb * 128) / 8 + sub] = codes;
+            if (COLS)
+                *reinterpret_cast<uint4 *>(&tile[row * 64 + sub * 4]) = v[p];
         }
-        if (COLS)
-            *reinterpret_cast<uint4 *>(&tile[row * 64 + sub * 4]) = v[p];
+    } else if (COLS) {
+#pragma unroll
+        for (int p = 0; p < 8; ++p)
+            *reinterpret_cast<uint4 *>(&tile[(p * 16 + rsub) * 64 + sub * 4]) = v[p];
     }
     if (COLS) {
         __syncthreads();
@@ -454,11 +519,12 @@ quant_tile_kernel(const uint4 *__restrict__ x, int64_t M, int64_t K, uint2 *__re
                 chi[i / 4] |= cvt_e4m3x2(a.y, b.y) << (16 * ((i / 2) & 1));
             }
         } else if (dlo.fast && dhi.fast) {
-            const float2 r2 = make_float2(dlo.r, dhi.r), ns2 = make_float2(-s_lo, -s_hi);
+            const float2 r2 = make_float2(dlo.r, dhi.r), nr2 = make_float2(-dlo.r, -dhi.r);
+            const float2 s2 = make_float2(s_lo, s_hi);
 #pragma unroll
             for (int i = 0; i < 32; i += 2) {
-                const float2 a = div2_fast(make_float2(bf16lo(w[i]), bf16hi(w[i])), r2, ns2);
-                const float2 b = div2_fast(make_float2(bf16lo(w[i + 1]), bf16hi(w[i + 1])), r2, ns2);
+                const float2 a = div2_fast(make_float2(bf16lo(w[i]), bf16hi(w[i])), r2, nr2, s2);
+                const float2 b = div2_fast(make_float2(bf16lo(w[i + 1]), bf16hi(w[i + 1])), r2, nr2, s2);
                 clo[i / 4] |= cvt_e4m3x2(a.x, b.x) << (16 * ((i / 2) & 1));
                 chi[i / 4] |= cvt_e4m3x2(a.y, b.y) << (16 * ((i / 2) & 1));
             }
