@@ -8,8 +8,8 @@ There is no CPU fallback: if the library is missing or the device is not sm_100,
 the calls raise.
 
 Method (Puro-2B, part 3/7, section 3.2 "FP8 Mixed-Precision Training"): E4M3
-operands, one scale per 128 consecutive values along the GEMM reduction dimension
-for activations and activation gradients, one per 128x128 block for weights, FP32
+operands; activations and their gradients scaled per 128 neighbouring elements in
+the summed (K) direction, weights per 128x128 tile; FP32
 scales amax/448, and fprop / dgrad / wgrad GEMMs in FP8 with a BF16 result.
 """
 from __future__ import annotations

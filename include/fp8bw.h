@@ -5,9 +5,9 @@
  * The operations follow Puro-2B ("Poor Lab's Qwen2-1.5B Trained on RTX 5090 within
  * $5090", arXiv HTML part 3/7), section 3.2 "FP8 Mixed-Precision Training":
  * Transformer linear layers quantize their BF16 inputs and weights to E4M3
- * immediately before each GEMM, with one scale per 128 consecutive values along the
- * GEMM reduction dimension for activations and activation gradients and one scale
- * per 128x128 block for weights; fprop, dgrad and wgrad all run in FP8 and the layer
+ * immediately before each GEMM.  Activations and their gradients carry a scale for
+ * every 128 neighbouring elements in the direction the GEMM sums over, weights a
+ * scale for every 128x128 tile; fprop, dgrad and wgrad all run in FP8 and the layer
  * hands a BF16 result back to the model.  Each block scale is the block's absolute
  * maximum divided by 448 (the largest finite E4M3 magnitude) in FP32, and values are
  * divided by it and rounded to nearest-even onto E4M3, saturating at +-448 (the
@@ -62,9 +62,9 @@ typedef enum { FP8BW_FPROP = 0, FP8BW_DGRAD = 1, FP8BW_WGRAD = 2 } fp8bw_mode;
 #define FP8BW_MAX_DIM (1 << 20)
 
 /*
- * fp8_quant_act -- 1x128 groups along the reduction dimension (section 3.2:
- * "activations and activation gradients use one-dimensional groups of 128
- * consecutive values along the GEMM reduction dimension").
+ * fp8_quant_act -- 1x128 groups along the reduction dimension (section 3.2: the
+ * scales of activations and of their gradients are taken over runs of 128 adjacent
+ * elements in the direction the GEMM sums over).
  *   x  [M][K] BF16 in      q [M][K] E4M3 codes out      s [K/128][M] FP32 out
  * For each row m and block kb: amax = max |x[m][kb*128 .. kb*128+127]|,
  * s[kb][m] = amax / 448 (binary32 division), q = e4m3_rne_sat(x / s) with the
@@ -88,9 +88,9 @@ int fp8_quant_act_t(const void *x_bf16, int64_t M, int64_t K, uint8_t *qt, float
 
 /*
  * fp8_quant_act_dual -- both activation layouts from one read of X (section 3.2:
- * the layer's quantized input is retained for wgrad; this produces, in one pass over
- * the BF16 tensor, the row-wise copy fprop/dgrad consume and the token-wise copy
- * wgrad consumes).  Outputs are bit-identical to fp8_quant_act(x, M, K, q, s) and
+ * wgrad reuses the FP8 copy of the layer input made for fprop; this call produces,
+ * in one pass over the BF16 tensor, the row-wise copy fprop/dgrad consume and the
+ * token-wise copy wgrad consumes).  Outputs are bit-identical to fp8_quant_act(x, M, K, q, s) and
  * fp8_quant_act_t(x, M, K, qt, st):
  *   x [M][K] BF16 in
  *   q [M][K], s [K/128][M]      1x128 groups along K
@@ -100,8 +100,8 @@ int fp8_quant_act_dual(const void *x_bf16, int64_t M, int64_t K, uint8_t *q, flo
                        uint8_t *qt, float *st, void *stream);
 
 /*
- * fp8_quant_weight -- 128x128 blocks (section 3.2: "weights use two-dimensional
- * 128x128 blocks").
+ * fp8_quant_weight -- 128x128 blocks (section 3.2: a weight's scales are taken
+ * over square 128x128 tiles).
  *   w  [N][K] BF16 in      q [N][K] E4M3 out      s [N/128][K/128] FP32 out
  *   qt_or_null: if not NULL, also writes qt [K][N] = q transposed (same codes; a
  *   128x128 block keeps its one scale under transposition).
@@ -114,8 +114,9 @@ int fp8_quant_weight(const void *w_bf16, int64_t N, int64_t K, uint8_t *q, float
  * reduction cut into 128-long blocks kb.  For each kb the FP8 partial product
  * sum_{k in kb} qa*qb is accumulated in FP32 by the tensor cores and then promoted
  * into an FP32 running sum multiplied by (a-scale x b-scale) of that block; the sum
- * is rounded to BF16 (nearest-even) at the end.  Section 3.2: "their Fprop, Dgrad,
- * and Wgrad GEMMs all use the FP8 path", with a BF16 output for the model.
+ * is rounded to BF16 (nearest-even) at the end.  Section 3.2: the forward, input-gradient
+ * and weight-gradient GEMMs of these layers all run in FP8, with a BF16 output
+ * for the model.
  *
  *   FPROP  Y  = X . W^T   a = Qx  [M][K], sa = [K/128][M]   (from fp8_quant_act(X))
  *                         b = Qw  [N][K], sb = [N/128][K/128] (from fp8_quant_weight(W))

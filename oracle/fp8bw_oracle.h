@@ -9,12 +9,13 @@
  * $5090", part 3/7, section 3.2 "FP8 Mixed-Precision Training"):
  *   - Transformer linear operands are E4M3 (the FP8 format of Micikevicius et al.,
  *     "FP8 Formats for Deep Learning", 2022, cited there).
- *   - Activations and activation gradients get one scale per 128 consecutive
- *     values along the GEMM reduction dimension; weights one scale per 128x128 block.
+ *   - Activations and their gradients carry one scale for every 128 neighbouring
+ *     elements in the summed (K) direction; weights one scale per 128x128 tile.
  *   - The scales are computed online from the tensor being quantized.  The block
  *     scale is FP32 absmax/448 with saturating round-to-nearest-even onto E4M3,
  *     the DeepSeek-V3 fine-grained recipe that section 3.2 says it follows.
- *   - Fprop, dgrad and wgrad GEMMs all consume the FP8 operands and produce BF16.
+ *   - The forward, input-gradient and weight-gradient GEMMs each take FP8 operands
+ *     and return BF16.
  *
  * Layouts (row-major [rows][cols]):
  *   x, w          : BF16 bit patterns (uint16_t)
