@@ -281,11 +281,12 @@ int fp8bw_last_device_error(void *stream)
     int st;
     if (device_sms({}, &st) < 0)
         return st;
-    int v = 0, w = 0;
+    int v = 0, w = 0, u = 0;
     if (fp8bw::read_and_clear_device_error(static_cast<cudaStream_t>(stream), &v) != cudaSuccess ||
-        fp8bw::read_and_clear_mx_error(&w) != cudaSuccess)
+        fp8bw::read_and_clear_mx_error(&w) != cudaSuccess ||
+        fp8bw::read_and_clear_quant_error(&u) != cudaSuccess)
         return FP8BW_ECUDA;
-    return (v || w) ? FP8BW_ETIMEOUT : FP8BW_OK;
+    return (v || w || u) ? FP8BW_ETIMEOUT : FP8BW_OK;
 }
 
 int fp8bw_selftest_wait_timeout(int64_t limit_us, void *stream)

@@ -7,11 +7,14 @@
 // quotient rounded to FP32, then rounded to nearest-even onto E4M3 with saturation
 // at +-448 (cvt.rn.satfinite).  An all-zero group gets scale 0 and codes 0x00.
 //
-// All three kernels are HBM-bound streaming kernels: 2 bytes read and 1 + 4/128
-// bytes written per element.
+// Both kernels (the tile quantizer for activations, the block quantizer for weights)
+// are HBM-bound streaming kernels: 2 bytes read and 1 + 4/128 bytes written per
+// element and layout.
 #include <cstdint>
+#include <cuda.h>
 #include <cuda_runtime.h>
 
+#include "ptx.cuh"
 #include "quant.cuh"
 
 namespace fp8bw {
@@ -152,141 +155,6 @@ __device__ __forceinline__ uint2 quant8_pow2(uint4 v, float mul)
     return make_uint2(c[0] | (c[1] << 16), c[2] | (c[3] << 16));
 }
 
-// ------------------------------------------------------------ fp8_quant_act
-
-// A warp quantizes two consecutive groups at a time (half-warp h takes group
-// 2p + h); each lane holds 8 consecutive values (16 bytes).  Groups are enumerated
-// in memory order, g = m*(K/128) + kb, so the warps in flight stream through one
-// contiguous region of X and Q; the scale of group (m, kb) goes to s[kb][m].
-constexpr int QA_THREADS = 256;
-constexpr int QA_UNROLL = 4;
-
-__global__ void __launch_bounds__(QA_THREADS)
-quant_act_kernel(const uint4 *__restrict__ x, int64_t M, int64_t K, uint2 *__restrict__ q,
-                 float *__restrict__ s)
-{
-    const int64_t npairs = M * (K / 128) / 2;
-    const int64_t warp = (int64_t(blockIdx.x) * QA_THREADS + threadIdx.x) >> 5;
-    const int64_t nwarps = (int64_t(gridDim.x) * QA_THREADS) >> 5;
-    const int lane = threadIdx.x & 31;
-    const int half = lane >> 4, sub = lane & 15;
-
-    for (int64_t p0 = warp; p0 < npairs; p0 += nwarps * QA_UNROLL) {
-        uint4 v[QA_UNROLL];
-        int64_t off[QA_UNROLL];
-#pragma unroll
-        for (int u = 0; u < QA_UNROLL; ++u) {
-            int64_t p = p0 + int64_t(u) * nwarps;
-            off[u] = -1;
-            if (p < npairs) {
-                off[u] = (2 * p + half) * 16 + sub;  // in units of 8 elements
-                v[u] = __ldg(x + off[u]);
-            }
-        }
-#pragma unroll
-        for (int u = 0; u < QA_UNROLL; ++u) {
-            int64_t p = p0 + int64_t(u) * nwarps;
-            if (p >= npairs)  // uniform across the warp
-                break;
-            uint32_t m2 = __vmaxu2(absmax2(v[u].x, v[u].y), absmax2(v[u].z, v[u].w));
-#pragma unroll
-            for (int o = 8; o >= 1; o >>= 1)
-                m2 = __vmaxu2(m2, __shfl_xor_sync(0xffffffffu, m2, o));
-            float amax = halves_max_to_float(m2);
-            float sc = __fdiv_rn(amax, 448.0f);
-            uint2 codes = make_uint2(0u, 0u);
-            if (amax != 0.0f)
-                codes = quant8(v[u], GroupDiv(sc));
-            q[off[u]] = codes;
-            if (sub == 0) {
-                const int64_t g = 2 * p + half, KB = K / 128;
-                int64_t m, kb;
-                if (g < INT32_MAX) {  // 32-bit division in the common case
-                    const uint32_t g32 = uint32_t(g), kb32 = uint32_t(KB);
-                    m = g32 / kb32;
-                    kb = g32 - uint32_t(m) * kb32;
-                } else {
-                    m = g / KB;
-                    kb = g - m * KB;
-                }
-                s[kb * M + m] = sc;
-            }
-        }
-    }
-}
-
-// ---------------------------------------------------------- fp8_quant_act_t
-
-// Block tile: 128 rows (one token block mb) x 64 columns.  Warp w holds rows
-// 16w .. 16w+15; lane l holds columns 2l and 2l+1 of every one of those rows.
-// Column absmax: per lane over its 16 rows, then across the 8 warps in shared
-// memory.  Each lane then owns 16 consecutive tokens of two columns, which are 16
-// contiguous bytes of the transposed output: one 16-byte store per column.
-constexpr int QT_THREADS = 256;
-
-__global__ void __launch_bounds__(QT_THREADS)
-quant_act_t_kernel(const uint32_t *__restrict__ x, int64_t M, int64_t K,
-                   uint8_t *__restrict__ qt, float *__restrict__ st)
-{
-    __shared__ uint32_t red[8][32];
-    const int w = threadIdx.x >> 5, l = threadIdx.x & 31;
-    const int64_t k0 = int64_t(blockIdx.x) * 64;
-    const int64_t mb = blockIdx.y;
-    const int64_t row0 = mb * 128 + 16 * w;
-
-    uint32_t v[16];
-#pragma unroll
-    for (int r = 0; r < 16; ++r)
-        v[r] = __ldg(x + ((row0 + r) * K + k0) / 2 + l);
-    uint32_t m2 = 0;
-#pragma unroll
-    for (int r = 0; r < 16; r += 2)
-        m2 = __vmaxu2(m2, absmax2(v[r], v[r + 1]));
-    red[w][l] = m2;
-    __syncthreads();
-#pragma unroll
-    for (int i = 0; i < 8; ++i)
-        m2 = __vmaxu2(m2, red[i][l]);
-
-    const float amax_lo = __uint_as_float((m2 & 0xFFFFu) << 16);
-    const float amax_hi = __uint_as_float(m2 & 0xFFFF0000u);
-    const float s_lo = __fdiv_rn(amax_lo, 448.0f);
-    const float s_hi = __fdiv_rn(amax_hi, 448.0f);
-
-    // Lane values: v[r] holds (column 2l, column 2l+1) of row r, whose groups have
-    // the scales s_lo and s_hi, so each packed pair divides by a packed scale pair.
-    uint32_t clo[4] = {0u, 0u, 0u, 0u}, chi[4] = {0u, 0u, 0u, 0u};
-    const GroupDiv dlo(s_lo), dhi(s_hi);
-    if (dlo.fast && dhi.fast) {
-        const float2 r2 = make_float2(dlo.r, dhi.r), nr2 = make_float2(-dlo.r, -dhi.r);
-        const float2 s2 = make_float2(s_lo, s_hi);
-#pragma unroll
-        for (int r = 0; r < 16; r += 2) {
-            const float2 a = div2_fast(make_float2(bf16lo(v[r]), bf16hi(v[r])), r2, nr2, s2);
-            const float2 b = div2_fast(make_float2(bf16lo(v[r + 1]), bf16hi(v[r + 1])), r2, nr2, s2);
-            clo[r / 4] |= cvt_e4m3x2(a.x, b.x) << (16 * ((r / 2) & 1));
-            chi[r / 4] |= cvt_e4m3x2(a.y, b.y) << (16 * ((r / 2) & 1));
-        }
-    } else {
-#pragma unroll
-        for (int r = 0; r < 16; r += 2) {
-            clo[r / 4] |= cvt_e4m3x2(__fdiv_rn(bf16lo(v[r]), s_lo), __fdiv_rn(bf16lo(v[r + 1]), s_lo))
-                          << (16 * ((r / 2) & 1));
-            chi[r / 4] |= cvt_e4m3x2(__fdiv_rn(bf16hi(v[r]), s_hi), __fdiv_rn(bf16hi(v[r + 1]), s_hi))
-                          << (16 * ((r / 2) & 1));
-        }
-    }
-    if (amax_lo == 0.0f)
-        clo[0] = clo[1] = clo[2] = clo[3] = 0u;
-    if (amax_hi == 0.0f)
-        chi[0] = chi[1] = chi[2] = chi[3] = 0u;
-    const int64_t col = k0 + 2 * l;
-    *reinterpret_cast<uint4 *>(qt + col * M + row0) = make_uint4(clo[0], clo[1], clo[2], clo[3]);
-    *reinterpret_cast<uint4 *>(qt + (col + 1) * M + row0) = make_uint4(chi[0], chi[1], chi[2], chi[3]);
-    if (w == 0)
-        *reinterpret_cast<float2 *>(st + mb * K + col) = make_float2(s_lo, s_hi);
-}
-
 // --------------------------------------------------------- fp8_quant_weight
 
 // One block per 128x128 weight block.  Thread t covers, in each of 8 passes, row
@@ -369,57 +237,76 @@ quant_weight_kernel(const uint4 *__restrict__ w, int64_t N, int64_t K, uint2 *__
     }
 }
 
-// ------------------------------------------------------- tile quantizer (dual)
+// ------------------------------------------------------------ tile quantizer
 
-// One CTA per 128 x 128 tile of X (one reduction block of 128 rows).  Every thread
-// first loads its 8 x 16 bytes (rows t/16 + 16p, columns 8*(t%16) .. +7), so a CTA
-// has its whole 32 KB tile in flight before any arithmetic.
-//   ROWS: 1x128 groups along K (the tile's columns) -> q[M][K], s[K/128][M]; each
-//         half-warp holds one row, reduced with a 16-lane shuffle.
-//   COLS: 1x128 groups along M (the tile's rows) -> qt[K][M], st[M/128][K]; the tile
-//         goes through shared memory, thread t takes column pair t%64 over rows
-//         32*(t/64) .. +31 (conflict-free 4-byte reads), the four row quarters meet
-//         in shared memory for the column absmax.
+// One CTA per 128 x 128 tile of X (one reduction block of 128 rows).  One thread
+// brings the whole tile (32 KB of BF16) into shared memory with a single TMA load,
+// row-major: 256 bytes per row, the layout the token-wise transpose reads.  No thread
+// holds in-flight loads in registers, so five CTAs (five tiles' loads) share an SM.
+//   ROWS: 1x128 groups along K (the tile's columns) -> q[M][K], s[K/128][M].  Half-warp
+//         h of warp w holds rows 16p + 2w + h (p < 8), 8 values per lane: each lane's
+//         partial amax for its 8 rows goes through a transposing reduction over the
+//         16 lanes (recursive halving: exchange half of the rows' partials with the
+//         lane 8, 4, 2 apart, then combine with the lane 1 apart), after which lanes
+//         2p and 2p + 1 hold the amax of row 16p + rsub.  Each lane works out that one
+//         group's scale (and reciprocal), and the quantizing loop fetches group p's
+//         scalars by shuffle, so the per-group division and reciprocal run once per
+//         lane for all 8 groups instead of once per group.
+//   COLS: 1x128 groups along M (the tile's rows) -> qt[K][M], st[M/128][K]; thread t
+//         takes column pair t%64 over rows 32*(t/64) .. +31 (conflict-free 4-byte
+//         reads), the four row quarters meet in shared memory for the column absmax,
+//         and a second sweep quantizes.
 // With both, X is read once for the two layouts wgrad and fprop/dgrad need.
-constexpr int QD_THREADS = 256;
-
 // E8: power-of-two scales in 512-byte blocks (see sf_block_off): s holds
 // [M/128][K/128] blocks (row m of block (m/128, kb)), st holds [K/128][M/128] blocks
 // (column k of X is row k % 128 of block (k/128, mb)).
-// Four CTAs per SM (at most 64 registers): more tiles' loads in flight per SM.
-#ifndef FP8BW_QD_MINB
-#define FP8BW_QD_MINB 4
-#endif
+constexpr int QD_THREADS = 256;
+constexpr int QD_MIN_BLOCKS = 5;  // at most 48 registers
+
+__device__ int g_quant_error;  // first error code of a bounded wait in the quantizers
+constexpr int QERR_TILE_LOAD = 21;
+constexpr uint64_t QT_WAIT_NS = 1000000000ull;
+constexpr uint64_t QT_DRAIN_NS = 20000000ull;
+
 template <bool ROWS, bool COLS, bool E8 = false>
-__global__ void __launch_bounds__(QD_THREADS, FP8BW_QD_MINB)
-quant_tile_kernel(const uint4 *__restrict__ x, int64_t M, int64_t K, uint2 *__restrict__ q,
-                  void *__restrict__ s_out, uint8_t *__restrict__ qt, void *__restrict__ st_out)
+__global__ void __launch_bounds__(QD_THREADS, QD_MIN_BLOCKS)
+quant_tile_kernel(const __grid_constant__ CUtensorMap tmX, int64_t M, int64_t K,
+                      uint2 *__restrict__ q, void *__restrict__ s_out, uint8_t *__restrict__ qt,
+                      void *__restrict__ st_out)
 {
-    __shared__ uint32_t tile[COLS ? 128 * 64 : 1];
+    __shared__ __align__(128) uint32_t tile[128 * 64];
     __shared__ uint32_t red[4][64];
+    __shared__ uint64_t bar;
+    __shared__ int abort_flag;
     const int t = threadIdx.x;
     const int64_t kb = blockIdx.x, mb = blockIdx.y;
     const int rsub = t >> 4, sub = t & 15;
 
-    uint4 v[8];
-#pragma unroll
-    for (int p = 0; p < 8; ++p) {
-        const int64_t m = mb * 128 + p * 16 + rsub;
-        v[p] = __ldg(x + (m * K + kb * 128) / 8 + sub);
+    if (t == 0) {
+        mbar_init(&bar, 1);
+        abort_flag = 0;
+        fence_mbarrier_init();
+        mbar_arrive_expect_tx(&bar, 128 * 128 * 2);
+        tma_load_2d(tile, &tmX, &bar, int32_t(kb * 128), int32_t(mb * 128));
     }
+    __syncthreads();
+    if (!mbar_wait_bounded(&bar, 0u, &abort_flag, &g_quant_error, QERR_TILE_LOAD, QT_WAIT_NS)) {
+        if (t == 0) {  // keep the CTA (and its shared memory) alive while the copy may land
+            const uint64_t t0 = global_timer_ns();
+            while (global_timer_ns() - t0 < QT_DRAIN_NS) {
+            }
+        }
+        return;
+    }
+    const uint4 *tile4 = reinterpret_cast<const uint4 *>(tile);  // [128 rows][16 uint4]
+
     if (ROWS) {
-        // Row groups: half-warp h holds rows 16p + rsub (p < 8), 8 values per lane.
-        // Each lane's partial amax for its 8 rows goes through a transposing reduction
-        // over the 16 lanes (recursive halving: exchange half of the rows' partials with
-        // the lane 8, 4, 2 apart, then combine with the lane 1 apart), after which
-        // lanes 2p and 2p + 1 hold the amax of row 16p + rsub.  Each lane then works out
-        // the scale of that one group, and the quantizing loop fetches group p's
-        // scalars by shuffle: the per-group division and reciprocal run once per lane
-        // for all 8 groups instead of once per group.
         uint32_t mx[8];
 #pragma unroll
-        for (int p = 0; p < 8; ++p)
-            mx[p] = __vmaxu2(absmax2(v[p].x, v[p].y), absmax2(v[p].z, v[p].w));
+        for (int p = 0; p < 8; ++p) {
+            const uint4 v = tile4[(p * 16 + rsub) * 16 + sub];
+            mx[p] = __vmaxu2(absmax2(v.x, v.y), absmax2(v.z, v.w));
+        }
         {
             const bool b = (sub & 8) != 0;
 #pragma unroll
@@ -444,8 +331,6 @@ quant_tile_kernel(const uint4 *__restrict__ x, int64_t M, int64_t K, uint2 *__re
         mx[0] = __vmaxu2(mx[0], __shfl_xor_sync(0xffffffffu, mx[0], 1));
         const float amax = halves_max_to_float(mx[0]);
         const int64_t m_own = mb * 128 + (sub >> 1) * 16 + rsub;
-        // per group: E8 the multiplier 2^-e (0 for an all-zero group); FP32 the scale
-        // (0 for an all-zero group) and RN(1/s), or -1 when the group takes IEEE division
         float g0 = 0.0f, g1 = 0.0f;
         if constexpr (E8) {
             const int e = e8m0_exponent(amax);
@@ -463,38 +348,30 @@ quant_tile_kernel(const uint4 *__restrict__ x, int64_t M, int64_t K, uint2 *__re
         }
 #pragma unroll
         for (int p = 0; p < 8; ++p) {
-            const int row = p * 16 + rsub;
-            const int64_t m = mb * 128 + row;
+            const int64_t m = mb * 128 + p * 16 + rsub;
             const float gp = __shfl_sync(0xffffffffu, g0, 2 * p, 16);
+            const uint4 v = tile4[(p * 16 + rsub) * 16 + sub];
             uint2 codes = make_uint2(0u, 0u);
             if constexpr (E8) {
                 if (gp != 0.0f)
-                    codes = quant8_pow2(v[p], gp);
+                    codes = quant8_pow2(v, gp);
             } else {
                 const float rp = __shfl_sync(0xffffffffu, g1, 2 * p, 16);
                 if (gp != 0.0f)
-                    codes = rp > 0.0f ? quant8_fast(v[p], rp, gp) : quant8_ieee(v[p], gp);
+                    codes = rp > 0.0f ? quant8_fast(v, rp, gp) : quant8_ieee(v, gp);
             }
             q[(m * K + kb * 128) / 8 + sub] = codes;
-            if (COLS)
-                *reinterpret_cast<uint4 *>(&tile[row * 64 + sub * 4]) = v[p];
         }
-    } else if (COLS) {
-#pragma unroll
-        for (int p = 0; p < 8; ++p)
-            *reinterpret_cast<uint4 *>(&tile[(p * 16 + rsub) * 64 + sub * 4]) = v[p];
     }
     if (COLS) {
-        __syncthreads();
+        // Token groups: thread t takes column pair t % 64 over rows 32 (t / 64) .. +31;
+        // a first sweep for the column amax, a second to quantize.
         const int cp = t & 63, rq = t >> 6;
-        uint32_t w[32];
-#pragma unroll
-        for (int i = 0; i < 32; ++i)
-            w[i] = tile[(rq * 32 + i) * 64 + cp];
+        const uint32_t *col = tile + (rq * 32) * 64 + cp;
         uint32_t m2 = 0;
 #pragma unroll
         for (int i = 0; i < 32; i += 2)
-            m2 = __vmaxu2(m2, absmax2(w[i], w[i + 1]));
+            m2 = __vmaxu2(m2, absmax2(col[i * 64], col[(i + 1) * 64]));
         red[rq][cp] = m2;
         __syncthreads();
         m2 = __vmaxu2(__vmaxu2(red[0][cp], red[1][cp]), __vmaxu2(red[2][cp], red[3][cp]));
@@ -513,8 +390,9 @@ quant_tile_kernel(const uint4 *__restrict__ x, int64_t M, int64_t K, uint2 *__re
             const float2 mul2 = make_float2(pow2_neg(e_lo), pow2_neg(e_hi));
 #pragma unroll
             for (int i = 0; i < 32; i += 2) {
-                const float2 a = __fmul2_rn(make_float2(bf16lo(w[i]), bf16hi(w[i])), mul2);
-                const float2 b = __fmul2_rn(make_float2(bf16lo(w[i + 1]), bf16hi(w[i + 1])), mul2);
+                const uint32_t w0 = col[i * 64], w1 = col[(i + 1) * 64];
+                const float2 a = __fmul2_rn(make_float2(bf16lo(w0), bf16hi(w0)), mul2);
+                const float2 b = __fmul2_rn(make_float2(bf16lo(w1), bf16hi(w1)), mul2);
                 clo[i / 4] |= cvt_e4m3x2(a.x, b.x) << (16 * ((i / 2) & 1));
                 chi[i / 4] |= cvt_e4m3x2(a.y, b.y) << (16 * ((i / 2) & 1));
             }
@@ -523,19 +401,19 @@ quant_tile_kernel(const uint4 *__restrict__ x, int64_t M, int64_t K, uint2 *__re
             const float2 s2 = make_float2(s_lo, s_hi);
 #pragma unroll
             for (int i = 0; i < 32; i += 2) {
-                const float2 a = div2_fast(make_float2(bf16lo(w[i]), bf16hi(w[i])), r2, nr2, s2);
-                const float2 b = div2_fast(make_float2(bf16lo(w[i + 1]), bf16hi(w[i + 1])), r2, nr2, s2);
+                const uint32_t w0 = col[i * 64], w1 = col[(i + 1) * 64];
+                const float2 a = div2_fast(make_float2(bf16lo(w0), bf16hi(w0)), r2, nr2, s2);
+                const float2 b = div2_fast(make_float2(bf16lo(w1), bf16hi(w1)), r2, nr2, s2);
                 clo[i / 4] |= cvt_e4m3x2(a.x, b.x) << (16 * ((i / 2) & 1));
                 chi[i / 4] |= cvt_e4m3x2(a.y, b.y) << (16 * ((i / 2) & 1));
             }
         } else {
 #pragma unroll
             for (int i = 0; i < 32; i += 2) {
-                clo[i / 4] |= cvt_e4m3x2(__fdiv_rn(bf16lo(w[i]), s_lo),
-                                         __fdiv_rn(bf16lo(w[i + 1]), s_lo))
+                const uint32_t w0 = col[i * 64], w1 = col[(i + 1) * 64];
+                clo[i / 4] |= cvt_e4m3x2(__fdiv_rn(bf16lo(w0), s_lo), __fdiv_rn(bf16lo(w1), s_lo))
                               << (16 * ((i / 2) & 1));
-                chi[i / 4] |= cvt_e4m3x2(__fdiv_rn(bf16hi(w[i]), s_hi),
-                                         __fdiv_rn(bf16hi(w[i + 1]), s_hi))
+                chi[i / 4] |= cvt_e4m3x2(__fdiv_rn(bf16hi(w0), s_hi), __fdiv_rn(bf16hi(w1), s_hi))
                               << (16 * ((i / 2) & 1));
             }
         }
@@ -549,75 +427,97 @@ quant_tile_kernel(const uint4 *__restrict__ x, int64_t M, int64_t K, uint2 *__re
             for (int i = 0; i < 8; ++i)
                 chi[i] = 0u;
         }
-        const int64_t col = kb * 128 + 2 * cp;
+        const int64_t c = kb * 128 + 2 * cp;
         const int64_t m0 = mb * 128 + rq * 32;
-        uint4 *dlo_p = reinterpret_cast<uint4 *>(qt + col * M + m0);
-        uint4 *dhi_p = reinterpret_cast<uint4 *>(qt + (col + 1) * M + m0);
+        uint4 *dlo_p = reinterpret_cast<uint4 *>(qt + c * M + m0);
+        uint4 *dhi_p = reinterpret_cast<uint4 *>(qt + (c + 1) * M + m0);
         dlo_p[0] = make_uint4(clo[0], clo[1], clo[2], clo[3]);
         dlo_p[1] = make_uint4(clo[4], clo[5], clo[6], clo[7]);
         dhi_p[0] = make_uint4(chi[0], chi[1], chi[2], chi[3]);
         dhi_p[1] = make_uint4(chi[4], chi[5], chi[6], chi[7]);
         if (rq == 0) {
             if (E8) {
-                uint8_t *blk = static_cast<uint8_t *>(st_out) + ((col >> 7) * (M / 128) + mb) * 512;
-                *reinterpret_cast<uint32_t *>(blk + sf_block_off(int(col & 127))) = rep4_code(e_lo, amax_lo);
-                *reinterpret_cast<uint32_t *>(blk + sf_block_off(int((col + 1) & 127))) = rep4_code(e_hi, amax_hi);
+                uint8_t *blk = static_cast<uint8_t *>(st_out) + ((c >> 7) * (M / 128) + mb) * 512;
+                *reinterpret_cast<uint32_t *>(blk + sf_block_off(int(c & 127))) = rep4_code(e_lo, amax_lo);
+                *reinterpret_cast<uint32_t *>(blk + sf_block_off(int((c + 1) & 127))) = rep4_code(e_hi, amax_hi);
             } else
-                *reinterpret_cast<float2 *>(static_cast<float *>(st_out) + mb * K + col) =
+                *reinterpret_cast<float2 *>(static_cast<float *>(st_out) + mb * K + c) =
                     make_float2(s_lo, s_hi);
         }
     }
 }
 
+typedef CUresult (*QEncodeFn)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *,
+                              const cuuint64_t *, const cuuint64_t *, const cuuint32_t *,
+                              const cuuint32_t *, CUtensorMapInterleave, CUtensorMapSwizzle,
+                              CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+// BF16 [M][K] map with 128 x 128 boxes, no swizzle (rows of 256 bytes).
+static bool tile_map_bf16(CUtensorMap *map, const void *x, int64_t M, int64_t K)
+{
+    static QEncodeFn enc = [] {
+        void *p = nullptr;
+        cudaDriverEntryPointQueryResult r;
+        if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &p, 12000, cudaEnableDefault,
+                                             &r) != cudaSuccess ||
+            r != cudaDriverEntryPointSuccess)
+            p = nullptr;
+        return reinterpret_cast<QEncodeFn>(p);
+    }();
+    if (!enc)
+        return false;
+    cuuint64_t gdim[2] = {cuuint64_t(K), cuuint64_t(M)};
+    cuuint64_t gstride[1] = {cuuint64_t(K) * 2};
+    cuuint32_t box[2] = {128, 128};
+    cuuint32_t estride[2] = {1, 1};
+    return enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(x), gdim, gstride, box,
+               estride, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+               CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+template <bool ROWS, bool COLS, bool E8>
+static cudaError_t run_tile(const void *x, int64_t M, int64_t K, void *q, void *s, uint8_t *qt,
+                                void *st, cudaStream_t stream)
+{
+    CUtensorMap map;
+    if (!tile_map_bf16(&map, x, M, K))
+        return cudaErrorInvalidValue;
+    dim3 grid(unsigned(K / 128), unsigned(M / 128));
+    quant_tile_kernel<ROWS, COLS, E8><<<grid, QD_THREADS, 0, stream>>>(
+        map, M, K, reinterpret_cast<uint2 *>(q), s, qt, st);
+    return cudaGetLastError();
+}
+
+cudaError_t read_and_clear_quant_error(int *value)
+{
+    cudaError_t e = cudaMemcpyFromSymbol(value, g_quant_error, sizeof(int));
+    if (e != cudaSuccess)
+        return e;
+    if (*value) {
+        const int zero = 0;
+        e = cudaMemcpyToSymbol(g_quant_error, &zero, sizeof(int));
+    }
+    return e;
+}
+
 // ------------------------------------------------------------------ launchers
 
-#ifndef FP8BW_QUANT_TILE
-#define FP8BW_QUANT_TILE 1
-#endif
-
 cudaError_t launch_quant_act(const void *x, int64_t M, int64_t K, uint8_t *q, float *s,
-                             cudaStream_t stream, int num_sms)
+                             cudaStream_t stream, int /*num_sms*/)
 {
-    if (FP8BW_QUANT_TILE) {
-        dim3 grid(unsigned(K / 128), unsigned(M / 128));
-        quant_tile_kernel<true, false><<<grid, QD_THREADS, 0, stream>>>(
-            static_cast<const uint4 *>(x), M, K, reinterpret_cast<uint2 *>(q), s, nullptr,
-            nullptr);
-        return cudaGetLastError();
-    }
-    const int64_t npairs = M * (K / 128) / 2;
-    const int64_t warps_needed = (npairs + QA_UNROLL - 1) / QA_UNROLL;
-    int64_t blocks = (warps_needed + (QA_THREADS / 32) - 1) / (QA_THREADS / 32);
-    const int64_t cap = int64_t(num_sms) * 8;
-    if (blocks > cap)
-        blocks = cap;
-    quant_act_kernel<<<dim3(unsigned(blocks)), QA_THREADS, 0, stream>>>(
-        static_cast<const uint4 *>(x), M, K, reinterpret_cast<uint2 *>(q), s);
-    return cudaGetLastError();
+    return run_tile<true, false, false>(x, M, K, q, s, nullptr, nullptr, stream);
 }
 
 cudaError_t launch_quant_dual(const void *x, int64_t M, int64_t K, uint8_t *q, float *s,
                               uint8_t *qt, float *st, cudaStream_t stream)
 {
-    dim3 grid(unsigned(K / 128), unsigned(M / 128));
-    quant_tile_kernel<true, true><<<grid, QD_THREADS, 0, stream>>>(
-        static_cast<const uint4 *>(x), M, K, reinterpret_cast<uint2 *>(q), s, qt, st);
-    return cudaGetLastError();
+    return run_tile<true, true, false>(x, M, K, q, s, qt, st, stream);
 }
 
 cudaError_t launch_quant_act_t(const void *x, int64_t M, int64_t K, uint8_t *qt, float *st,
                                cudaStream_t stream)
 {
-    if (FP8BW_QUANT_TILE) {
-        dim3 grid(unsigned(K / 128), unsigned(M / 128));
-        quant_tile_kernel<false, true><<<grid, QD_THREADS, 0, stream>>>(
-            static_cast<const uint4 *>(x), M, K, nullptr, nullptr, qt, st);
-        return cudaGetLastError();
-    }
-    dim3 grid(unsigned(K / 64), unsigned(M / 128));
-    quant_act_t_kernel<<<grid, QT_THREADS, 0, stream>>>(static_cast<const uint32_t *>(x), M, K,
-                                                       qt, st);
-    return cudaGetLastError();
+    return run_tile<false, true, false>(x, M, K, nullptr, nullptr, qt, st, stream);
 }
 
 cudaError_t launch_quant_weight(const void *w, int64_t N, int64_t K, uint8_t *q, float *s,
@@ -634,27 +534,20 @@ cudaError_t launch_quant_weight(const void *w, int64_t N, int64_t K, uint8_t *q,
 cudaError_t launch_quant_e8m0(int which, const void *x, int64_t M, int64_t K, uint8_t *q,
                               uint8_t *s, uint8_t *qt, uint8_t *st, cudaStream_t stream)
 {
-    dim3 grid(unsigned(K / 128), unsigned(M / 128));
-    const uint4 *xv = static_cast<const uint4 *>(x);
-    uint2 *qv = reinterpret_cast<uint2 *>(q);
     switch (which) {
     case 0:  // rows: q[M][K], s[K/128][M]
-        quant_tile_kernel<true, false, true><<<grid, QD_THREADS, 0, stream>>>(xv, M, K, qv, s,
-                                                                            nullptr, nullptr);
-        break;
+        return run_tile<true, false, true>(x, M, K, q, s, nullptr, nullptr, stream);
     case 1:  // token groups: qt[K][M], st[M/128][K]
-        quant_tile_kernel<false, true, true><<<grid, QD_THREADS, 0, stream>>>(xv, M, K, nullptr,
-                                                                            nullptr, qt, st);
-        break;
+        return run_tile<false, true, true>(x, M, K, nullptr, nullptr, qt, st, stream);
     case 2:  // both
-        quant_tile_kernel<true, true, true><<<grid, QD_THREADS, 0, stream>>>(xv, M, K, qv, s, qt,
-                                                                           st);
-        break;
-    default:  // weight blocks: q[N=M][K], s[M/128][K/128], optional qt[K][M]
-        quant_weight_kernel<true><<<grid, QW_THREADS, 0, stream>>>(xv, M, K, qv, s, qt);
-        break;
+        return run_tile<true, true, true>(x, M, K, q, s, qt, st, stream);
+    default: {  // weight blocks: q[N=M][K], s[M/128][K/128], optional qt[K][M]
+        dim3 grid(unsigned(K / 128), unsigned(M / 128));
+        quant_weight_kernel<true><<<grid, QW_THREADS, 0, stream>>>(
+            static_cast<const uint4 *>(x), M, K, reinterpret_cast<uint2 *>(q), s, qt);
+        return cudaGetLastError();
     }
-    return cudaGetLastError();
+    }
 }
 
 } // namespace fp8bw

@@ -17,6 +17,9 @@ cudaError_t launch_quant_dual(const void *x, int64_t M, int64_t K, uint8_t *q, f
 cudaError_t launch_quant_e8m0(int which, const void *x, int64_t M, int64_t K, uint8_t *q,
                               uint8_t *s, uint8_t *qt, uint8_t *st, cudaStream_t stream);
 
+// Error word of the quantizers' bounded waits (read and cleared; caller synchronizes).
+cudaError_t read_and_clear_quant_error(int *value);
+
 cudaError_t launch_quant_weight(const void *w, int64_t N, int64_t K, uint8_t *q, float *s,
                                 uint8_t *qt, cudaStream_t stream);
 
