@@ -30,13 +30,13 @@
  *                distinct streams may run concurrently from different threads.
  *   Errors       Every call returns an fp8bw_status and never aborts or throws.
  *                Argument errors are reported before anything is launched.  A failed
- *                launch returns FP8BW_ECUDA.  The GEMM bounds every wait inside the
- *                kernel; a wait that runs out sets a per-device error word that
- *                fp8bw_last_device_error() reads.
+ *                launch returns FP8BW_ECUDA.  The GEMMs and the activation quantizers
+ *                bound every wait inside their kernels; a wait that runs out sets a
+ *                per-device error word that fp8bw_last_device_error() reads.
  *   Inputs       Finite BF16 values.  Non-finite inputs give unspecified codes but
  *                never fault.
- *   Memory       The library allocates no device memory: the per-device error word
- *                is a static device variable and TMA descriptors are passed by value.
+ *   Memory       The library allocates no device memory: the per-device error words
+ *                are static device variables and TMA descriptors are passed by value.
  */
 #ifndef FP8BW_H
 #define FP8BW_H
@@ -199,7 +199,8 @@ const char *fp8bw_status_string(int status);
 
 /* Synchronizes `stream`, then reads and clears the current device's error word:
  * FP8BW_OK, or FP8BW_ETIMEOUT if a bounded in-kernel wait ran out since the last
- * call (the GEMM whose wait ran out returned early and its output is undefined). */
+ * call (the GEMM or quantizer whose wait ran out returned early and its output is
+ * undefined). */
 int fp8bw_last_device_error(void *stream);
 
 /* Self-test of the failure-detection path (no counterpart in the paper; it checks
