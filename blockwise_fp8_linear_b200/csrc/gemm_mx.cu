@@ -327,18 +327,15 @@ fp8_gemm_mx_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constan
             uint32_t packed[COLS / 2];
 #pragma unroll
             for (int c = 0; c < COLS / 64; ++c) {
-                uint32_t v0[32], v1[32];
-                tmem_ld_32x32b_x32(taddr + uint32_t(64 * c), v0);
-                tmem_ld_32x32b_x32(taddr + uint32_t(64 * c + 32), v1);
+                // one 64-column TMEM load per chunk (fewer, larger tcgen05.ld)
+                uint32_t v[64];
+                tmem_ld_32x32b_x64(taddr + uint32_t(64 * c), v);
                 tmem_wait_ld();
 #pragma unroll
-                for (int e = 0; e < 16; ++e) {
-                    __nv_bfloat162 h0 = __floats2bfloat162_rn(__uint_as_float(v0[2 * e]),
-                                                              __uint_as_float(v0[2 * e + 1]));
-                    __nv_bfloat162 h1 = __floats2bfloat162_rn(__uint_as_float(v1[2 * e]),
-                                                              __uint_as_float(v1[2 * e + 1]));
-                    packed[32 * c + e] = *reinterpret_cast<uint32_t *>(&h0);
-                    packed[32 * c + 16 + e] = *reinterpret_cast<uint32_t *>(&h1);
+                for (int e = 0; e < 32; ++e) {
+                    __nv_bfloat162 h = __floats2bfloat162_rn(__uint_as_float(v[2 * e]),
+                                                             __uint_as_float(v[2 * e + 1]));
+                    packed[32 * c + e] = *reinterpret_cast<uint32_t *>(&h);
                 }
             }
             // the accumulator is in registers: hand it back to the MMA issuer
