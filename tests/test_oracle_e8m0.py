@@ -154,3 +154,25 @@ def test_fp32_and_power_of_two_scales_on_a_gemm():
     r32, r8 = rel(y32), rel(y8)
     assert r32 < 0.05 and r8 < 0.05
     assert r8 >= 0.9 * r32
+
+
+@pytest.mark.parametrize("pos", [(0, 0), (0, 127), (77, 3), (127, 127)])
+def test_weight_scale_is_the_whole_blocks_amax(pos):
+    """Puro-2B part 3/7, section 3.2: a weight's scale covers its 128x128 tile, so the
+    exponent follows the tile's largest magnitude wherever it sits; the planted
+    element lands exactly on +-448 and every other code is the exact nearest value
+    of x / 2^e."""
+    rng = np.random.default_rng(5)
+    w = rng.uniform(-1.0, 1.0, size=(128, 256))
+    i, j = pos
+    w[i, 128 + j] = -3584.0                     # 448 * 2^3, exactly representable in BF16
+    bits = synth.f64_to_bf16_bits(w)
+    q, s, _ = oracle.quant_weight_e8m0(bits)
+    assert int(s[0, 1]) == 3 + 127
+    assert q[i, 128 + j] == 0xFE                 # -448
+    amax0 = max(abs(_bf16_value(int(b))) for b in bits[:, :128].ravel())
+    assert int(s[0, 0]) == _exact_exponent(amax0) + 127
+    for r in (0, i, 127):
+        for c in (0, j, 127):
+            v = bf16_to_fraction(int(bits[r, 128 + c]))
+            assert int(q[r, 128 + c]) == nearest_e4m3(v[0] / 8, v[1])
