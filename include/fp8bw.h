@@ -115,8 +115,8 @@ int fp8_quant_weight(const void *w_bf16, int64_t N, int64_t K, uint8_t *q, float
  * sum_{k in kb} qa*qb is accumulated in FP32 by the tensor cores and then promoted
  * into an FP32 running sum multiplied by (a-scale x b-scale) of that block; the sum
  * is rounded to BF16 (nearest-even) at the end.  Section 3.2: the forward, input-gradient
- * and weight-gradient GEMMs of these layers all run in FP8, with a BF16 output
- * for the model.
+ * and weight-gradient GEMMs of these layers all run in FP8, and the model receives
+ * BF16 results.
  *
  *   FPROP  Y  = X . W^T   a = Qx  [M][K], sa = [K/128][M]   (from fp8_quant_act(X))
  *                         b = Qw  [N][K], sb = [N/128][K/128] (from fp8_quant_weight(W))
