@@ -27,7 +27,9 @@ flush is needed between steps.
 
 Usage:  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
 Under torchrun (N > 1) each rank runs an independent replica (weak scaling): the path
-shards by tokens with no exchange in the data path.
+shards by tokens with no exchange in the data path.  --dp-grad reduce-scatter adds the
+data-parallel weight-gradient exchange: each linear's dW is reduce-scattered by rows
+over NCCL on the stream that computed it, overlapping the next linear's kernels.
 """
 from __future__ import annotations
 
