@@ -28,8 +28,9 @@ flush is needed between steps.
 Usage:  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
 Under torchrun (N > 1) each rank runs an independent replica (weak scaling): the path
 shards by tokens with no exchange in the data path.  --dp-grad reduce-scatter adds the
-data-parallel weight-gradient exchange: each linear's dW is reduce-scattered by rows
-over NCCL on the stream that computed it, overlapping the next linear's kernels.
+data-parallel weight-gradient exchange: each linear's wgrad accumulates into an FP32
+main gradient (fp8_gemm_wgrad_acc32), which is reduce-scattered by rows over NCCL on
+the stream that computed it, overlapping the next linear's kernels.
 """
 from __future__ import annotations
 
@@ -55,6 +56,12 @@ LINEARS = [("qkv", 2048, 4096), ("o", 2048, 2048), ("gate_up", 2048, 12288), ("d
 WORKLOAD = "qwen3-1.7b block linears (qkv, o, gate_up, down) fprop+dgrad+wgrad, M=8192"
 STEP_FLOPS = sum(3 * 2 * TOKENS * din * dout for _, din, dout in LINEARS)
 FP8_OVER_BF16 = 4.5 / 2.25  # nominal dense FP8 : BF16 tensor throughput on B200
+NOMINAL_FP8_TFLOPS = 4500.0  # B200 dense FP8 tensor peak as NVIDIA states it
+NOMINAL_HBM_GBS = 8000.0     # B200 HBM3e bandwidth as NVIDIA states it (DGX figure)
+# algorithmic bytes per element: BF16 read + per layout (E4M3 code + FP32 scale / 128)
+DUAL_BYTES = 2 + 2 * (1 + 4 / 128)
+ACT_BYTES = 2 + 1 + 4 / 128
+WEIGHT_BYTES = 2 + 1 + 4 / (128 * 128)  # one FP32 scale per 128x128 block
 
 
 def config_dict(n, overlap=True, dp_grad=False):
@@ -67,7 +74,8 @@ def config_dict(n, overlap=True, dp_grad=False):
         "passes": "fprop+dgrad+wgrad with all quantizers (X and dY quantized once into both layouts)",
         "step_gflop": round(STEP_FLOPS / 1e9, 3),
         "l2": "inputs larger than L2 (637 MB of BF16 inputs per step), no flush",
-        "parallelism": (f"dp{n}, dW reduce-scatter (NCCL) overlapped with the next linear" if dp_grad
+        "parallelism": (f"dp{n}, FP32 main-grad (wgrad_acc32) reduce-scatter over NCCL, "
+                        "overlapped with the next linear" if dp_grad
                         else f"replicas x{n}" if n > 1 else "single GPU"),
     }
 
@@ -215,9 +223,10 @@ class LayerWork:
         self.h2d_bytes = sum(d[k].numel() * 2 for d in self.lin for k in ("X", "W", "dY"))
         self.d2h_bytes = sum(d[k].numel() * 2 for d in self.lin for k in ("Y", "dX", "dW"))
 
-    def step(self, gemm_events=None, side=None, hooks=None, reducer=None):
+    def step(self, gemm_events=None, side=None, hooks=None, reducer=None, quant_events=None):
         """Enqueue one step on the current stream.  gemm_events: optional list that
-        receives (start, end, flops) CUDA-event triples around each GEMM.  side: an
+        receives (start, end, flops) CUDA-event triples around each GEMM; quant_events:
+        likewise (start, end, kind, shape, bytes) around each quantizer.  side: an
         optional second stream; each linear's wgrad then runs there, after the dY
         quantizer and concurrently with the dgrad (the two are independent given
         dY), and the current stream waits for it at the end of the step.
@@ -254,6 +263,16 @@ class LayerWork:
             if rc:
                 raise fb.Fp8bwError(rc, what)
 
+        def quant(fn, args, kind, shape, nbytes):
+            if quant_events is not None:
+                e0 = torch.cuda.Event(enable_timing=True)
+                e1 = torch.cuda.Event(enable_timing=True)
+                e0.record(main)
+            chk(fn(*args), kind)
+            if quant_events is not None:
+                e1.record(main)
+                quant_events.append((e0, e1, kind, shape, nbytes))
+
         for i, d in enumerate(self.lin):
             din, dout = d["din"], d["dout"]
             if hooks is not None:
@@ -261,16 +280,19 @@ class LayerWork:
             if self.separate:
                 chk(q_act(d["X"].data_ptr(), T, din, d["qx"].data_ptr(), d["sx"].data_ptr(), st), "qa")
             else:  # X read once: row-wise copy for fprop, token-wise copy kept for wgrad
-                chk(q_dual(d["X"].data_ptr(), T, din, d["qx"].data_ptr(), d["sx"].data_ptr(),
-                           d["qxt"].data_ptr(), d["sxt"].data_ptr(), st), "qd")
-            chk(q_weight(d["W"].data_ptr(), dout, din, d["qw"].data_ptr(),
-                         d["sw"].data_ptr(), None, st), "qw")
+                quant(q_dual, (d["X"].data_ptr(), T, din, d["qx"].data_ptr(), d["sx"].data_ptr(),
+                               d["qxt"].data_ptr(), d["sxt"].data_ptr(), st),
+                      "quant_act_dual", (T, din), T * din * DUAL_BYTES)
+            quant(q_weight, (d["W"].data_ptr(), dout, din, d["qw"].data_ptr(),
+                             d["sw"].data_ptr(), None, st),
+                  "quant_weight", (dout, din), dout * din * WEIGHT_BYTES)
             gemm(fb.FPROP, d["qx"], d["sx"], d["qw"], d["sw"], d["Y"], T, dout, din)
             if self.separate:
                 chk(q_act(d["dY"].data_ptr(), T, dout, d["qdy"].data_ptr(), d["sdy"].data_ptr(), st), "qa")
             else:
-                chk(q_dual(d["dY"].data_ptr(), T, dout, d["qdy"].data_ptr(), d["sdy"].data_ptr(),
-                           d["qdyt"].data_ptr(), d["sdyt"].data_ptr(), st), "qd")
+                quant(q_dual, (d["dY"].data_ptr(), T, dout, d["qdy"].data_ptr(), d["sdy"].data_ptr(),
+                               d["qdyt"].data_ptr(), d["sdyt"].data_ptr(), st),
+                      "quant_act_dual", (T, dout), T * dout * DUAL_BYTES)
             if self.separate:
                 chk(q_act_t(d["dY"].data_ptr(), T, dout, d["qdyt"].data_ptr(), d["sdyt"].data_ptr(), st), "qt")
                 chk(q_act_t(d["X"].data_ptr(), T, din, d["qxt"].data_ptr(), d["sxt"].data_ptr(), st), "qt")
@@ -281,9 +303,22 @@ class LayerWork:
                 ready.record(main)
                 side.wait_event(ready)
             gemm(fb.DGRAD, d["qdy"], d["sdy"], d["qw"], d["sw"], d["dX"], T, din, dout)
-            gemm(fb.WGRAD, d["qdyt"], d["sdyt"], d["qxt"], d["sxt"], d["dW"], dout, din, T, stream=side)
-            if reducer is not None:
-                reducer.launch(i, d["dW"], side if side is not None else main)
+            if reducer is None:
+                gemm(fb.WGRAD, d["qdyt"], d["sdyt"], d["qxt"], d["sxt"], d["dW"], dout, din, T,
+                     stream=side)
+            else:
+                # data-parallel step: this rank's token reduction accumulates into the
+                # FP32 main gradient, which is then summed over the ranks (reduce-scatter)
+                ws = side if side is not None else main
+                dw32 = d.setdefault("dW32", torch.empty(dout, din, dtype=torch.float32,
+                                                        device=d["dW"].device))
+                with torch.cuda.stream(ws):
+                    dw32.zero_()
+                chk(L.fp8_gemm_wgrad_acc32(d["qdyt"].data_ptr(), d["sdyt"].data_ptr(),
+                                           d["qxt"].data_ptr(), d["sxt"].data_ptr(),
+                                           dw32.data_ptr(), dout, din, T, ws.cuda_stream),
+                    "wgrad_acc32")
+                reducer.launch(i, dw32, ws)
             if hooks is not None:
                 hooks.after(i, main, side if side is not None else main)
         if side is not None:
@@ -306,41 +341,6 @@ def make_inputs(rank=0):
     return out
 
 
-class DpGradReducer:
-    """Data-parallel weight-gradient exchange: each linear's dW [out][in] is summed over
-    the ranks and split by rows, rank r keeping rows [r*out/N, (r+1)*out/N) (a
-    reduce-scatter, the gradient layout of an optimizer sharded by rows).  On GPUs the
-    collective is NCCL over NVLink, issued on the stream that computed dW so that it
-    overlaps the next linear's kernels; wait() makes the current stream wait for all
-    of them.  CPU tensors and the gloo backend take the same path (for tests)."""
-
-    def __init__(self, shapes, world, device):
-        import torch
-        self.world = world
-        self.shards = [torch.empty(dout // world, din, dtype=torch.bfloat16, device=device)
-                       for dout, din in shapes]
-        self.pending = []
-
-    @staticmethod
-    def rows(dout, world, rank):
-        return rank * dout // world, (rank + 1) * dout // world
-
-    def launch(self, i, dW, stream=None):
-        import torch
-        import torch.distributed as dist
-        if stream is not None:
-            with torch.cuda.stream(stream):
-                h = dist.reduce_scatter_tensor(self.shards[i], dW, op=dist.ReduceOp.SUM, async_op=True)
-        else:
-            h = dist.reduce_scatter_tensor(self.shards[i], dW, op=dist.ReduceOp.SUM, async_op=True)
-        self.pending.append(h)
-
-    def wait(self):
-        for h in self.pending:
-            h.wait()
-        self.pending.clear()
-
-
 def barrier(world):
     if world > 1:
         import torch.distributed as dist
@@ -357,6 +357,86 @@ def max_over_ranks(x, world):
     t = torch.tensor([x], dtype=torch.float64, device=dev)
     dist.all_reduce(t, op=dist.ReduceOp.MAX)
     return float(t.item())
+
+
+def gemm_summary(gemm_events, work):
+    """Mean device time and TFLOP/s of each of the step's 12 GEMMs (linear x mode) over
+    the one-stream pass (events in launch order: per linear fprop, dgrad, wgrad)."""
+    names = [(d["name"], m) for d in work.lin for m in ("fprop", "dgrad", "wgrad")]
+    acc = {}
+    for j, (e0, e1, f) in enumerate(gemm_events):
+        key = names[j % len(names)]
+        t, ff, n = acc.get(key, (0.0, 0.0, 0))
+        acc[key] = (t + e0.elapsed_time(e1), ff + f, n + 1)
+    return [{"gemm": f"{k[0]}_{k[1]}", "us": round(1e3 * t / n, 2),
+             "tflops": round(ff / (t * 1e-3) / 1e12, 1)} for k, (t, ff, n) in acc.items()]
+
+
+def quant_summary(quant_events):
+    """GB/s of each quantizer kind and shape (algorithmic bytes / mean device time)."""
+    acc = {}
+    for e0, e1, kind, shape, nbytes in quant_events:
+        key = (kind, tuple(shape))
+        t, b, n = acc.get(key, (0.0, 0.0, 0))
+        acc[key] = (t + e0.elapsed_time(e1), b + nbytes, n + 1)
+    return [{"kernel": k, "shape": list(shp), "launches": n, "us": round(1e3 * t / n, 2),
+             "gbs": round(b / (t * 1e-3) / 1e9, 1)} for (k, shp), (t, b, n) in sorted(acc.items())]
+
+
+def single_fprop_latency(dev, reps=200):
+    """The single-fprop workload (X[128][1024] ~ N(0,1), W[1024][1024] ~ N(0,0.02),
+    seed 0) through the C ABI: fp8_quant_act(X), fp8_quant_weight(W) and the FPROP
+    GEMM.  Latency-bound, so it is reported in microseconds: device time per layer
+    call (events around `reps` calls back to back) and per GEMM alone, plus the host
+    time to issue one layer call."""
+    import torch
+    import blockwise_fp8_linear_b200 as fb
+    from blockwise_fp8_linear_b200 import synth
+    L = fb.lib()
+    T, Din, Dout = 128, 1024, 1024
+    t = lambda a: torch.from_numpy(a.view(np.int16)).view(torch.bfloat16).to(dev)
+    X = t(synth.normal_bf16(T, Din, 1.0, seed=synth.seed_for(0, 0)))
+    W = t(synth.normal_bf16(Dout, Din, 0.02, seed=synth.seed_for(0, 1)))
+    qx = torch.empty(T, Din, dtype=torch.uint8, device=dev)
+    sx = torch.empty(Din // 128, T, dtype=torch.float32, device=dev)
+    qw = torch.empty(Dout, Din, dtype=torch.uint8, device=dev)
+    sw = torch.empty(Dout // 128, Din // 128, dtype=torch.float32, device=dev)
+    Y = torch.empty(T, Dout, dtype=torch.bfloat16, device=dev)
+    st = torch.cuda.current_stream().cuda_stream
+
+    def layer():
+        rc = (L.fp8_quant_act(X.data_ptr(), T, Din, qx.data_ptr(), sx.data_ptr(), st)
+              or L.fp8_quant_weight(W.data_ptr(), Dout, Din, qw.data_ptr(), sw.data_ptr(), None, st)
+              or L.fp8_gemm_blockwise(0, qx.data_ptr(), sx.data_ptr(), qw.data_ptr(),
+                                      sw.data_ptr(), Y.data_ptr(), T, Dout, Din, st))
+        if rc:
+            raise fb.Fp8bwError(rc, "single fprop")
+
+    def gemm():
+        rc = L.fp8_gemm_blockwise(0, qx.data_ptr(), sx.data_ptr(), qw.data_ptr(), sw.data_ptr(),
+                                  Y.data_ptr(), T, Dout, Din, st)
+        if rc:
+            raise fb.Fp8bwError(rc, "single fprop gemm")
+
+    out = {"workload": "single fprop linear: X[128x1024], W[1024x1024], Y = X W^T (bf16)",
+           "gflop": round(2 * T * Din * Dout / 1e9, 4)}
+    for name, fn in (("layer", layer), ("gemm", gemm)):
+        for _ in range(10):
+            fn()
+        torch.cuda.synchronize()
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        h0 = time.perf_counter()
+        e0.record()
+        for _ in range(reps):
+            fn()
+        e1.record()
+        h1 = time.perf_counter()
+        torch.cuda.synchronize()
+        out[f"{name}_us"] = round(1e3 * e0.elapsed_time(e1) / reps, 2)
+        out[f"{name}_host_issue_us"] = round(1e6 * (h1 - h0) / reps, 2)
+    out["unit"] = "us"
+    return out
 
 
 def run_ours(args):
@@ -378,6 +458,7 @@ def run_ours(args):
     side = None if args.no_overlap else torch.cuda.Stream(device=dev)
     reducer = None
     if world > 1 and args.dp_grad == "reduce-scatter":
+        from blockwise_fp8_linear_b200.dp import DpGradReducer
         reducer = DpGradReducer([(dout, din) for _, din, dout in LINEARS], world, dev)
 
     # warm-up
@@ -389,19 +470,20 @@ def run_ours(args):
 
     # kernel roofline: the same K steps on one stream, every GEMM launch bracketed by
     # events, so that each launch's time is its own (no overlap with another kernel)
-    gemm_events = []
+    gemm_events, quant_events = [], []
     barrier(world)
     torch.cuda.synchronize()
     r0 = torch.cuda.Event(enable_timing=True)
     r1 = torch.cuda.Event(enable_timing=True)
     r0.record()
     for _ in range(args.steps):
-        work.step(gemm_events)
+        work.step(gemm_events, quant_events=quant_events)
     r1.record()
     torch.cuda.synchronize()
     serial_ms = r0.elapsed_time(r1)
     gemm_ms = sum(e0.elapsed_time(e1) for e0, e1, _ in gemm_events)
     gemm_flops = sum(f for _, _, f in gemm_events)
+    quant_rows = quant_summary(quant_events)
 
     # timed region: K steps, device time by CUDA events on the launching stream
     with ClockSampler(dev.index) as clocks:
@@ -423,6 +505,29 @@ def run_ours(args):
 
     ms_per_step = elapsed_ms / args.steps
     value = world * STEP_FLOPS / (ms_per_step * 1e-3) / 1e12
+
+    # sustained: the same step repeated for a few seconds, deep into the power cap
+    sustained = None
+    if args.sustain_s > 0:
+        n_sus = max(args.steps, int(args.sustain_s * 1e3 / max(ms_per_step, 1e-3)))
+        n_sus = int(max_over_ranks(float(n_sus), world))
+        with ClockSampler(dev.index) as sclk:
+            barrier(world)
+            torch.cuda.synchronize()
+            s0 = torch.cuda.Event(enable_timing=True)
+            s1 = torch.cuda.Event(enable_timing=True)
+            s0.record()
+            for _ in range(n_sus):
+                work.step(side=side, reducer=reducer)
+            s1.record()
+            torch.cuda.synchronize()
+            barrier(world)
+        sus_ms = max_over_ranks(s0.elapsed_time(s1), world)
+        if fb.fp8bw_last_device_error() != 0:
+            raise RuntimeError("a bounded in-kernel wait ran out in the sustained run")
+        sustained = {"value": round(world * STEP_FLOPS / (sus_ms / n_sus * 1e-3) / 1e12, 3),
+                     "unit": UNIT, "ms_per_step": round(sus_ms / n_sus, 4), "steps": n_sus,
+                     "seconds": round(sus_ms / 1e3, 3), "clocks": sclk.summary()}
 
     # end to end through the public API: pinned host inputs -> device, step,
     # results -> pinned host, all inside the timed region
@@ -503,17 +608,36 @@ def run_ours(args):
 
     peaks, peak_src = measured_peaks()
     fp8_peak = peaks["bf16_tflops"] * FP8_OVER_BF16
+    hbm_peak = float(peaks["hbm_gbs"])
     achieved = gemm_flops / (gemm_ms * 1e-3) / 1e12
     roofline = {
         "kernel": "fp8_gemm_kernel (fprop/dgrad/wgrad, all 12 GEMMs of the step)",
         "bound": "tensor", "achieved": round(achieved, 2),
         "peak": round(fp8_peak, 1), "unit": "TFLOP/s", "frac": round(achieved / fp8_peak, 4),
         "peak_source": f"{peak_src} cuBLAS bf16 burst x {FP8_OVER_BF16:g} (nominal FP8:BF16)",
+        "nominal_peak": NOMINAL_FP8_TFLOPS,
+        "frac_of_nominal": round(achieved / NOMINAL_FP8_TFLOPS, 4),
+        "target": ">= 0.60 of dense FP8 peak, reported against both the measured peak "
+                  "(frac) and the nominal 4.5 PFLOP/s (frac_of_nominal)",
         "traffic": recorded_traffic(),
         "traffic_unit": "bytes per GEMM launch (mean over the step's 12 GEMMs, ncu dram read+write)",
         "gemm_share_of_step": round(gemm_ms / serial_ms, 4),
         "measured_on": "a separate pass of the same steps on one stream (no kernel overlap)",
+        "per_gemm": gemm_summary(gemm_events, work),
     }
+    quant_roofline = {
+        "bound": "hbm", "unit": "GB/s", "peak": hbm_peak,
+        "peak_source": f"{peak_src} HBM copy bandwidth",
+        "nominal_peak": NOMINAL_HBM_GBS,
+        "target": ">= 0.75 of HBM bandwidth, reported against both the measured copy "
+                  "bandwidth (frac) and the nominal 8 TB/s (frac_of_nominal)",
+        "bytes_per_element": {"quant_act_dual": DUAL_BYTES, "quant_weight": WEIGHT_BYTES},
+        "measured_on": "the same one-stream pass, every quantizer launch bracketed by events",
+        "kernels": [dict(r, frac=round(r["gbs"] / hbm_peak, 4),
+                         frac_of_nominal=round(r["gbs"] / NOMINAL_HBM_GBS, 4))
+                    for r in quant_rows],
+    }
+    single = single_fprop_latency(dev) if not args.no_single else None
 
     # the same step with power-of-two (E8M0) scales applied by the block-scaled MMA
     # (the MXFP8 form of the recipe), for comparison; not the headline
@@ -528,14 +652,15 @@ def run_ours(args):
             work8.step(ev8)
         v0 = torch.cuda.Event(enable_timing=True)
         v1 = torch.cuda.Event(enable_timing=True)
-        barrier(world)
-        torch.cuda.synchronize()
-        v0.record()
-        for _ in range(args.steps):
-            work8.step(side=side)
-        v1.record()
-        torch.cuda.synchronize()
-        barrier(world)
+        with ClockSampler(dev.index) as vclk:
+            barrier(world)
+            torch.cuda.synchronize()
+            v0.record()
+            for _ in range(args.steps):
+                work8.step(side=side)
+            v1.record()
+            torch.cuda.synchronize()
+            barrier(world)
         if fb.fp8bw_last_device_error() != 0:
             raise RuntimeError("a bounded in-kernel wait ran out in the E8M0 variant")
         v_ms = max_over_ranks(v0.elapsed_time(v1), world) / args.steps
@@ -544,8 +669,9 @@ def run_ours(args):
         variant = {"scales": "e8m0 (power of two, scale blocks applied by tcgen05.mma block_scale)",
                    "value": round(world * STEP_FLOPS / (v_ms * 1e-3) / 1e12, 3), "unit": UNIT,
                    "ms_per_step": round(v_ms, 4), "gemm_tflops": round(g8, 2),
-                   "gemm_frac": round(g8 / (measured_peaks()[0]["bf16_tflops"] * FP8_OVER_BF16), 4),
-                   "gemm_kernel": "fp8_gemm_mx_kernel"}
+                   "gemm_frac": round(g8 / fp8_peak, 4),
+                   "gemm_frac_of_nominal": round(g8 / NOMINAL_FP8_TFLOPS, 4),
+                   "gemm_kernel": "fp8_gemm_mx_kernel", "clocks": vclk.summary()}
         del work8
 
     cpu = None
@@ -564,6 +690,10 @@ def run_ours(args):
             "e2e": e2e, "gpu_launches": work.launches_per_step * args.steps,
             "clocks": clock_info,
             "pct_of_fp8_peak": round(100 * value / world / fp8_peak, 2),
+            "pct_of_nominal_fp8_peak": round(100 * value / world / NOMINAL_FP8_TFLOPS, 2),
+            "quant_roofline": quant_roofline,
+            "single_fprop": single,
+            "sustained": sustained,
             "variant_e8m0": variant,
         }
         print(json.dumps(line), flush=True)
@@ -602,6 +732,19 @@ def oracle_sample_step(i, host, threads):
     return 2 * M * N * K, time.perf_counter() - t
 
 
+def cpu_model():
+    """The host CPU's model name (Linux /proc/cpuinfo), or the platform's processor string."""
+    try:
+        with open("/proc/cpuinfo") as f:
+            for line in f:
+                if line.lower().startswith("model name"):
+                    return line.split(":", 1)[1].strip()
+    except OSError:
+        pass
+    import platform
+    return platform.processor() or "unknown"
+
+
 def cpu_baseline(budget_s=15.0, host=None, max_steps=None):
     import oracle
     threads = oracle.max_threads()
@@ -616,7 +759,7 @@ def cpu_baseline(budget_s=15.0, host=None, max_steps=None):
         secs += s
         n += 1
     return {"value": round(flops / secs / 1e12, 6), "unit": UNIT, "cores": threads,
-            "kind": "oracle",
+            "cpu_model": cpu_model(), "nproc": os.cpu_count(), "kind": "oracle",
             "sample": f"{n} samples, each one 128-row output tile of one of the 12 GEMMs of the "
                       f"step (rotating linear x mode) plus the oracle quantization of the groups "
                       f"it reads; FP64 GEMM, {threads} OpenMP threads, {secs:.1f} s"}
@@ -644,7 +787,8 @@ def run_reference(args):
         "ms_per_step": round(1e3 * secs / args.steps, 3), "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
         "config": config_dict(world),
-        "cpu_baseline": {"value": round(value, 6), "unit": UNIT, "cores": threads, "kind": "oracle",
+        "cpu_baseline": {"value": round(value, 6), "unit": UNIT, "cores": threads,
+                         "cpu_model": cpu_model(), "nproc": os.cpu_count(), "kind": "oracle",
                          "sample": "each step: one 128-row output tile of one of the 12 GEMMs "
                                    "(rotating), with the quantization of the groups it reads"},
         "e2e": {"value": round(value, 6), "unit": UNIT, "h2d_bytes_per_step": 0,
@@ -863,6 +1007,11 @@ def main():
                          "linear's dW over the ranks (NCCL), overlapped with the next linear")
     ap.add_argument("--no-variant", action="store_true",
                     help="skip the power-of-two (E8M0) scale variant of the step")
+    ap.add_argument("--sustain-s", type=float, default=2.5,
+                    help="seconds of the same step repeated after the timed region, reported "
+                         "as 'sustained' (0 = skip)")
+    ap.add_argument("--no-single", action="store_true",
+                    help="skip the single-fprop latency measurement")
     ap.add_argument("--no-overlap", action="store_true",
                     help="run every kernel on one stream (no dgrad/wgrad overlap)")
     ap.add_argument("--kernel-only", choices=KERNEL_CASES, default=None,

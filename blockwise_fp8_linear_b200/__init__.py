@@ -99,14 +99,61 @@ def _check(status: int, what: str):
         raise Fp8bwError(status, what)
 
 
-def _need(t, dtype, ndim, name):
+def _validate(items):
+    """Check the tensor arguments of one call before anything reaches the C ABI.
+    items: (tensor or None, dtype, shape, name); None marks an output to allocate.
+    Shapes are checked first, for every tensor, then dtype, contiguity and that all
+    are CUDA tensors of one device.  A size that disagreed with the M, N, K handed to
+    the C call would let a kernel read or write past an allocation, so every mismatch
+    raises here (ValueError for shapes and devices, TypeError for kinds)."""
     import torch
-    if not isinstance(t, torch.Tensor) or not t.is_cuda:
-        raise TypeError(f"{name} must be a CUDA tensor")
-    if t.dtype != dtype:
-        raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
-    if t.dim() != ndim or not t.is_contiguous():
-        raise ValueError(f"{name} must be a contiguous {ndim}-D tensor")
+    given = [(t, dt, shp, name) for t, dt, shp, name in items if t is not None]
+    for t, _, shp, name in given:
+        if not isinstance(t, torch.Tensor):
+            raise TypeError(f"{name} must be a torch tensor")
+        if tuple(t.shape) != tuple(int(d) for d in shp):
+            raise ValueError(f"{name} has shape {tuple(t.shape)}, expected {tuple(shp)}")
+    for t, dt, _, name in given:
+        if t.dtype != dt:
+            raise TypeError(f"{name} must be {dt}, got {t.dtype}")
+        if not t.is_contiguous():
+            raise ValueError(f"{name} must be contiguous")
+        if not t.is_cuda:
+            raise TypeError(f"{name} must be a CUDA tensor")
+    dev = given[0][0].device
+    for t, _, _, name in given:
+        if t.device != dev:
+            raise ValueError(f"{name} is on {t.device}, expected {dev} (one device per call)")
+    return dev
+
+
+def _alloc(t, shape, dtype, device):
+    import torch
+    return torch.empty(shape, dtype=dtype, device=device) if t is None else t
+
+
+def _dims(M, N=None, K=None):
+    """Sizes must be positive multiples of 128 (the ABI rejects others; checked here
+    so that buffer shapes derived from them are whole)."""
+    for d in (M, N, K):
+        if d is not None and (int(d) <= 0 or int(d) % 128):
+            raise ValueError(f"size {d} is not a positive multiple of 128")
+
+
+def _on(device):
+    """Context that makes `device` current, so the call's stream and the current device
+    match its buffers (the ABI rejects buffers of another device)."""
+    import torch
+    return torch.cuda.device(device)
+
+
+def _x2(x, name):
+    import torch
+    if not isinstance(x, torch.Tensor) or x.dim() != 2:
+        raise ValueError(f"{name} must be a 2-D tensor")
+    M, K = x.shape
+    _dims(M, K)
+    return int(M), int(K)
 
 
 def fp8bw_last_device_error(stream=None) -> int:
@@ -123,67 +170,97 @@ def fp8bw_selftest_wait_timeout(limit_us: int, stream=None) -> None:
 def fp8_quant_act(x, q=None, s=None, stream=None):
     """X[M][K] bf16 -> (Q[M][K] uint8 E4M3 codes, S[K/128][M] float32)."""
     import torch
-    _need(x, torch.bfloat16, 2, "x")
-    M, K = x.shape
-    q = torch.empty((M, K), dtype=torch.uint8, device=x.device) if q is None else q
-    s = torch.empty((K // 128, M), dtype=torch.float32, device=x.device) if s is None else s
-    _check(lib().fp8_quant_act(x.data_ptr(), M, K, q.data_ptr(), s.data_ptr(), _stream(stream)),
-           "fp8_quant_act")
+    M, K = _x2(x, "x")
+    dev = _validate([(x, torch.bfloat16, (M, K), "x"), (q, torch.uint8, (M, K), "q"),
+                     (s, torch.float32, (K // 128, M), "s")])
+    q = _alloc(q, (M, K), torch.uint8, dev)
+    s = _alloc(s, (K // 128, M), torch.float32, dev)
+    with _on(dev):
+        _check(lib().fp8_quant_act(x.data_ptr(), M, K, q.data_ptr(), s.data_ptr(),
+                                   _stream(stream)), "fp8_quant_act")
     return q, s
 
 
 def fp8_quant_act_t(x, qt=None, st=None, stream=None):
     """X[M][K] bf16 -> (Q^T[K][M] uint8, S^T[M/128][K] float32), groups along M."""
     import torch
-    _need(x, torch.bfloat16, 2, "x")
-    M, K = x.shape
-    qt = torch.empty((K, M), dtype=torch.uint8, device=x.device) if qt is None else qt
-    st = torch.empty((M // 128, K), dtype=torch.float32, device=x.device) if st is None else st
-    _check(lib().fp8_quant_act_t(x.data_ptr(), M, K, qt.data_ptr(), st.data_ptr(),
-                                 _stream(stream)), "fp8_quant_act_t")
+    M, K = _x2(x, "x")
+    dev = _validate([(x, torch.bfloat16, (M, K), "x"), (qt, torch.uint8, (K, M), "qt"),
+                     (st, torch.float32, (M // 128, K), "st")])
+    qt = _alloc(qt, (K, M), torch.uint8, dev)
+    st = _alloc(st, (M // 128, K), torch.float32, dev)
+    with _on(dev):
+        _check(lib().fp8_quant_act_t(x.data_ptr(), M, K, qt.data_ptr(), st.data_ptr(),
+                                     _stream(stream)), "fp8_quant_act_t")
     return qt, st
 
 
 def fp8_quant_act_dual(x, q=None, s=None, qt=None, st=None, stream=None):
     """X[M][K] bf16 -> (Q, S, Q^T, S^T): both layouts from one read of X."""
     import torch
-    _need(x, torch.bfloat16, 2, "x")
-    M, K = x.shape
-    q = torch.empty((M, K), dtype=torch.uint8, device=x.device) if q is None else q
-    s = torch.empty((K // 128, M), dtype=torch.float32, device=x.device) if s is None else s
-    qt = torch.empty((K, M), dtype=torch.uint8, device=x.device) if qt is None else qt
-    st = torch.empty((M // 128, K), dtype=torch.float32, device=x.device) if st is None else st
-    _check(lib().fp8_quant_act_dual(x.data_ptr(), M, K, q.data_ptr(), s.data_ptr(), qt.data_ptr(),
-                                    st.data_ptr(), _stream(stream)), "fp8_quant_act_dual")
+    M, K = _x2(x, "x")
+    dev = _validate([(x, torch.bfloat16, (M, K), "x"), (q, torch.uint8, (M, K), "q"),
+                     (s, torch.float32, (K // 128, M), "s"), (qt, torch.uint8, (K, M), "qt"),
+                     (st, torch.float32, (M // 128, K), "st")])
+    q = _alloc(q, (M, K), torch.uint8, dev)
+    s = _alloc(s, (K // 128, M), torch.float32, dev)
+    qt = _alloc(qt, (K, M), torch.uint8, dev)
+    st = _alloc(st, (M // 128, K), torch.float32, dev)
+    with _on(dev):
+        _check(lib().fp8_quant_act_dual(x.data_ptr(), M, K, q.data_ptr(), s.data_ptr(),
+                                        qt.data_ptr(), st.data_ptr(), _stream(stream)),
+               "fp8_quant_act_dual")
     return q, s, qt, st
 
 
 def fp8_quant_weight(w, want_t: bool = False, q=None, s=None, qt=None, stream=None):
     """W[N][K] bf16 -> (Q[N][K] uint8, S[N/128][K/128] float32, Q^T[K][N] or None)."""
     import torch
-    _need(w, torch.bfloat16, 2, "w")
-    N, K = w.shape
-    q = torch.empty((N, K), dtype=torch.uint8, device=w.device) if q is None else q
-    s = torch.empty((N // 128, K // 128), dtype=torch.float32, device=w.device) if s is None else s
-    if want_t and qt is None:
-        qt = torch.empty((K, N), dtype=torch.uint8, device=w.device)
-    _check(lib().fp8_quant_weight(w.data_ptr(), N, K, q.data_ptr(), s.data_ptr(),
-                                  qt.data_ptr() if qt is not None else None, _stream(stream)),
-           "fp8_quant_weight")
+    N, K = _x2(w, "w")
+    dev = _validate([(w, torch.bfloat16, (N, K), "w"), (q, torch.uint8, (N, K), "q"),
+                     (s, torch.float32, (N // 128, K // 128), "s"),
+                     (qt, torch.uint8, (K, N), "qt")])
+    q = _alloc(q, (N, K), torch.uint8, dev)
+    s = _alloc(s, (N // 128, K // 128), torch.float32, dev)
+    if want_t:
+        qt = _alloc(qt, (K, N), torch.uint8, dev)
+    with _on(dev):
+        _check(lib().fp8_quant_weight(w.data_ptr(), N, K, q.data_ptr(), s.data_ptr(),
+                                      qt.data_ptr() if qt is not None else None,
+                                      _stream(stream)), "fp8_quant_weight")
     return q, s, qt
+
+
+def _gemm_shapes(mode: int, M: int, N: int, K: int, e8m0: bool = False):
+    """Operand shapes of each GEMM mode (include/fp8bw.h): a, sa, b, sb."""
+    if mode not in (FPROP, DGRAD, WGRAD):
+        raise ValueError(f"mode must be FPROP, DGRAD or WGRAD, got {mode}")
+    _dims(M, N, K)
+    a = (M, K)
+    b = (K, N) if mode == DGRAD else (N, K)
+    if not e8m0:
+        sa = (K // 128, M)
+        sb = {FPROP: (N // 128, K // 128), DGRAD: (K // 128, N // 128), WGRAD: (K // 128, N)}[mode]
+    else:  # 512-byte scale blocks, one per 128 rows x 128-deep reduction block
+        sa = (M // 128, (K // 128) * 512)
+        sb = (K // 128, (N // 128) * 512) if mode == DGRAD else (N // 128, (K // 128) * 512)
+    return a, sa, b, sb
 
 
 def fp8_gemm_blockwise(mode: int, a, sa, b, sb, M: int, N: int, K: int, out=None, stream=None):
     """D[M][N] bf16 from FP8 operands and blockwise scales; see include/fp8bw.h for the
     operand layouts of FPROP, DGRAD and WGRAD."""
     import torch
-    for t, dt, name in ((a, torch.uint8, "a"), (b, torch.uint8, "b"),
-                        (sa, torch.float32, "sa"), (sb, torch.float32, "sb")):
-        _need(t, dt, 2, name)
-    out = torch.empty((M, N), dtype=torch.bfloat16, device=a.device) if out is None else out
-    _check(lib().fp8_gemm_blockwise(int(mode), a.data_ptr(), sa.data_ptr(), b.data_ptr(),
-                                    sb.data_ptr(), out.data_ptr(), M, N, K, _stream(stream)),
-           "fp8_gemm_blockwise")
+    M, N, K = int(M), int(N), int(K)
+    sh_a, sh_sa, sh_b, sh_sb = _gemm_shapes(mode, M, N, K)
+    dev = _validate([(a, torch.uint8, sh_a, "a"), (sa, torch.float32, sh_sa, "sa"),
+                     (b, torch.uint8, sh_b, "b"), (sb, torch.float32, sh_sb, "sb"),
+                     (out, torch.bfloat16, (M, N), "out")])
+    out = _alloc(out, (M, N), torch.bfloat16, dev)
+    with _on(dev):
+        _check(lib().fp8_gemm_blockwise(int(mode), a.data_ptr(), sa.data_ptr(), b.data_ptr(),
+                                        sb.data_ptr(), out.data_ptr(), M, N, K, _stream(stream)),
+               "fp8_gemm_blockwise")
     return out
 
 
@@ -191,13 +268,17 @@ def fp8_gemm_wgrad_acc32(a, sa, b, sb, M: int, N: int, K: int, dw32, stream=None
     """dw32[M][N] (float32, caller-owned) += the wgrad sum, kept in FP32 (no BF16
     rounding); a, sa, b, sb as for fp8_gemm_blockwise(WGRAD, ...)."""
     import torch
-    for t, dt, name in ((a, torch.uint8, "a"), (b, torch.uint8, "b"),
-                        (sa, torch.float32, "sa"), (sb, torch.float32, "sb"),
-                        (dw32, torch.float32, "dw32")):
-        _need(t, dt, 2, name)
-    _check(lib().fp8_gemm_wgrad_acc32(a.data_ptr(), sa.data_ptr(), b.data_ptr(), sb.data_ptr(),
-                                      dw32.data_ptr(), M, N, K, _stream(stream)),
-           "fp8_gemm_wgrad_acc32")
+    M, N, K = int(M), int(N), int(K)
+    sh_a, sh_sa, sh_b, sh_sb = _gemm_shapes(WGRAD, M, N, K)
+    if dw32 is None:
+        raise TypeError("dw32 must be a caller-owned float32 tensor")
+    dev = _validate([(a, torch.uint8, sh_a, "a"), (sa, torch.float32, sh_sa, "sa"),
+                     (b, torch.uint8, sh_b, "b"), (sb, torch.float32, sh_sb, "sb"),
+                     (dw32, torch.float32, (M, N), "dw32")])
+    with _on(dev):
+        _check(lib().fp8_gemm_wgrad_acc32(a.data_ptr(), sa.data_ptr(), b.data_ptr(),
+                                          sb.data_ptr(), dw32.data_ptr(), M, N, K,
+                                          _stream(stream)), "fp8_gemm_wgrad_acc32")
     return dw32
 
 
@@ -207,54 +288,67 @@ def fp8_quant_act_e8m0(x, q=None, s=None, stream=None):
     """X[M][K] bf16 -> (Q[M][K] uint8, S: E8M0 scale blocks [M/128][(K/128)*512] uint8,
     the tensor-core layout described in include/fp8bw.h)."""
     import torch
-    _need(x, torch.bfloat16, 2, "x")
-    M, K = x.shape
-    q = torch.empty((M, K), dtype=torch.uint8, device=x.device) if q is None else q
-    s = torch.empty((M // 128, (K // 128) * 512), dtype=torch.uint8, device=x.device) if s is None else s
-    _check(lib().fp8_quant_act_e8m0(x.data_ptr(), M, K, q.data_ptr(), s.data_ptr(),
-                                    _stream(stream)), "fp8_quant_act_e8m0")
+    M, K = _x2(x, "x")
+    ssh = (M // 128, (K // 128) * 512)
+    dev = _validate([(x, torch.bfloat16, (M, K), "x"), (q, torch.uint8, (M, K), "q"),
+                     (s, torch.uint8, ssh, "s")])
+    q = _alloc(q, (M, K), torch.uint8, dev)
+    s = _alloc(s, ssh, torch.uint8, dev)
+    with _on(dev):
+        _check(lib().fp8_quant_act_e8m0(x.data_ptr(), M, K, q.data_ptr(), s.data_ptr(),
+                                        _stream(stream)), "fp8_quant_act_e8m0")
     return q, s
 
 
 def fp8_quant_act_t_e8m0(x, qt=None, st=None, stream=None):
     """X[M][K] bf16 -> (Q^T[K][M] uint8, S^T: E8M0 scale blocks [K/128][(M/128)*512])."""
     import torch
-    _need(x, torch.bfloat16, 2, "x")
-    M, K = x.shape
-    qt = torch.empty((K, M), dtype=torch.uint8, device=x.device) if qt is None else qt
-    st = torch.empty((K // 128, (M // 128) * 512), dtype=torch.uint8, device=x.device) if st is None else st
-    _check(lib().fp8_quant_act_t_e8m0(x.data_ptr(), M, K, qt.data_ptr(), st.data_ptr(),
-                                      _stream(stream)), "fp8_quant_act_t_e8m0")
+    M, K = _x2(x, "x")
+    tsh = (K // 128, (M // 128) * 512)
+    dev = _validate([(x, torch.bfloat16, (M, K), "x"), (qt, torch.uint8, (K, M), "qt"),
+                     (st, torch.uint8, tsh, "st")])
+    qt = _alloc(qt, (K, M), torch.uint8, dev)
+    st = _alloc(st, tsh, torch.uint8, dev)
+    with _on(dev):
+        _check(lib().fp8_quant_act_t_e8m0(x.data_ptr(), M, K, qt.data_ptr(), st.data_ptr(),
+                                          _stream(stream)), "fp8_quant_act_t_e8m0")
     return qt, st
 
 
-def fp8_quant_act_dual_e8m0(x, stream=None):
+def fp8_quant_act_dual_e8m0(x, q=None, s=None, qt=None, st=None, stream=None):
     """X[M][K] bf16 -> (Q, S, Q^T, S^T) with E8M0 scale codes, from one read of X."""
     import torch
-    _need(x, torch.bfloat16, 2, "x")
-    M, K = x.shape
-    dev = x.device
-    q = torch.empty((M, K), dtype=torch.uint8, device=dev)
-    s = torch.empty((M // 128, (K // 128) * 512), dtype=torch.uint8, device=dev)
-    qt = torch.empty((K, M), dtype=torch.uint8, device=dev)
-    st = torch.empty((K // 128, (M // 128) * 512), dtype=torch.uint8, device=dev)
-    _check(lib().fp8_quant_act_dual_e8m0(x.data_ptr(), M, K, q.data_ptr(), s.data_ptr(),
-                                         qt.data_ptr(), st.data_ptr(), _stream(stream)),
-           "fp8_quant_act_dual_e8m0")
+    M, K = _x2(x, "x")
+    ssh, tsh = (M // 128, (K // 128) * 512), (K // 128, (M // 128) * 512)
+    dev = _validate([(x, torch.bfloat16, (M, K), "x"), (q, torch.uint8, (M, K), "q"),
+                     (s, torch.uint8, ssh, "s"), (qt, torch.uint8, (K, M), "qt"),
+                     (st, torch.uint8, tsh, "st")])
+    q = _alloc(q, (M, K), torch.uint8, dev)
+    s = _alloc(s, ssh, torch.uint8, dev)
+    qt = _alloc(qt, (K, M), torch.uint8, dev)
+    st = _alloc(st, tsh, torch.uint8, dev)
+    with _on(dev):
+        _check(lib().fp8_quant_act_dual_e8m0(x.data_ptr(), M, K, q.data_ptr(), s.data_ptr(),
+                                             qt.data_ptr(), st.data_ptr(), _stream(stream)),
+               "fp8_quant_act_dual_e8m0")
     return q, s, qt, st
 
 
-def fp8_quant_weight_e8m0(w, want_t: bool = False, stream=None):
+def fp8_quant_weight_e8m0(w, want_t: bool = False, q=None, s=None, qt=None, stream=None):
     """W[N][K] bf16 -> (Q[N][K], S: E8M0 scale blocks [N/128][(K/128)*512], Q^T or None)."""
     import torch
-    _need(w, torch.bfloat16, 2, "w")
-    N, K = w.shape
-    q = torch.empty((N, K), dtype=torch.uint8, device=w.device)
-    s = torch.empty((N // 128, (K // 128) * 512), dtype=torch.uint8, device=w.device)
-    qt = torch.empty((K, N), dtype=torch.uint8, device=w.device) if want_t else None
-    _check(lib().fp8_quant_weight_e8m0(w.data_ptr(), N, K, q.data_ptr(), s.data_ptr(),
-                                       qt.data_ptr() if want_t else None, _stream(stream)),
-           "fp8_quant_weight_e8m0")
+    N, K = _x2(w, "w")
+    ssh = (N // 128, (K // 128) * 512)
+    dev = _validate([(w, torch.bfloat16, (N, K), "w"), (q, torch.uint8, (N, K), "q"),
+                     (s, torch.uint8, ssh, "s"), (qt, torch.uint8, (K, N), "qt")])
+    q = _alloc(q, (N, K), torch.uint8, dev)
+    s = _alloc(s, ssh, torch.uint8, dev)
+    if want_t:
+        qt = _alloc(qt, (K, N), torch.uint8, dev)
+    with _on(dev):
+        _check(lib().fp8_quant_weight_e8m0(w.data_ptr(), N, K, q.data_ptr(), s.data_ptr(),
+                                           qt.data_ptr() if qt is not None else None,
+                                           _stream(stream)), "fp8_quant_weight_e8m0")
     return q, s, qt
 
 
@@ -263,13 +357,16 @@ def fp8_gemm_blockwise_e8m0(mode: int, a, sa, b, sb, M: int, N: int, K: int, out
     """fp8_gemm_blockwise with E8M0 scale blocks (from the *_e8m0 quantizers), applied by
     the block-scaled MMA."""
     import torch
-    for t, dt, name in ((a, torch.uint8, "a"), (b, torch.uint8, "b"),
-                        (sa, torch.uint8, "sa"), (sb, torch.uint8, "sb")):
-        _need(t, dt, 2, name)
-    out = torch.empty((M, N), dtype=torch.bfloat16, device=a.device) if out is None else out
-    _check(lib().fp8_gemm_blockwise_e8m0(int(mode), a.data_ptr(), sa.data_ptr(), b.data_ptr(),
-                                         sb.data_ptr(), out.data_ptr(), M, N, K, _stream(stream)),
-           "fp8_gemm_blockwise_e8m0")
+    M, N, K = int(M), int(N), int(K)
+    sh_a, sh_sa, sh_b, sh_sb = _gemm_shapes(mode, M, N, K, e8m0=True)
+    dev = _validate([(a, torch.uint8, sh_a, "a"), (sa, torch.uint8, sh_sa, "sa"),
+                     (b, torch.uint8, sh_b, "b"), (sb, torch.uint8, sh_sb, "sb"),
+                     (out, torch.bfloat16, (M, N), "out")])
+    out = _alloc(out, (M, N), torch.bfloat16, dev)
+    with _on(dev):
+        _check(lib().fp8_gemm_blockwise_e8m0(int(mode), a.data_ptr(), sa.data_ptr(),
+                                             b.data_ptr(), sb.data_ptr(), out.data_ptr(), M, N, K,
+                                             _stream(stream)), "fp8_gemm_blockwise_e8m0")
     return out
 
 

@@ -14,13 +14,18 @@ constexpr int kMaxDevices = 64;
 std::atomic<int> g_sms[kMaxDevices];    // 0 = not queried yet, -1 = not sm_100
 std::atomic<int> g_major[kMaxDevices];
 
-// Makes the device that owns the buffers current for this thread and returns its
-// SM count, or -1 with *status set.  Every pointer must be device (or managed)
-// memory of one device: a host pointer would fault the kernel, so it is rejected
-// here (FP8BW_EINVAL).
+// Returns the SM count of the calling thread's current device, or -1 with *status
+// set.  Every pointer must be device (or managed) memory of the current device: a
+// host pointer would fault the kernel and another device's buffer would not match
+// the caller's stream, so both are rejected here (FP8BW_EINVAL).  The current
+// device is never changed.
 int device_sms(std::initializer_list<const void *> ptrs, int *status)
 {
-    int dev = -1;
+    int cur = -1;
+    if (cudaGetDevice(&cur) != cudaSuccess) {
+        *status = FP8BW_ECUDA;
+        return -1;
+    }
     for (const void *p : ptrs) {
         if (!p)
             continue;
@@ -34,23 +39,12 @@ int device_sms(std::initializer_list<const void *> ptrs, int *status)
             *status = FP8BW_EINVAL;
             return -1;
         }
-        if (dev >= 0 && at.device != dev) {
+        if (at.type == cudaMemoryTypeDevice && at.device != cur) {
             *status = FP8BW_EINVAL;
             return -1;
         }
-        dev = at.device;
     }
-    int cur = -1;
-    if (cudaGetDevice(&cur) != cudaSuccess) {
-        *status = FP8BW_ECUDA;
-        return -1;
-    }
-    if (dev < 0)
-        dev = cur;
-    if (dev != cur && cudaSetDevice(dev) != cudaSuccess) {
-        *status = FP8BW_ECUDA;
-        return -1;
-    }
+    const int dev = cur;
     if (dev >= kMaxDevices) {
         *status = FP8BW_ECUDA;
         return -1;

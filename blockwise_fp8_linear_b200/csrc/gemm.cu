@@ -39,6 +39,7 @@
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 
+#include "launch_cache.cuh"
 #include "ptx.cuh"
 #include "quant.cuh"
 
@@ -513,17 +514,15 @@ fp8_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__
                         }
                     }
                 } else if constexpr (Cfg::OUT32) {
+                    // Vector atomic adds (red.global.add.v4.f32): calls that overlap on the
+                    // same FP32 buffer only reorder their additions, as on the pair path.
                     float *dst = D32 + size_t(tm * Cfg::TILE_M + row_in_tile) * size_t(N) +
                                  size_t(tn * BN + col0);
 #pragma unroll
-                    for (int c = 0; c < COLS / 4; ++c) {
-                        float4 o = *reinterpret_cast<const float4 *>(dst + 4 * c);
-                        o.x += acc[2 * c].x;
-                        o.y += acc[2 * c].y;
-                        o.z += acc[2 * c + 1].x;
-                        o.w += acc[2 * c + 1].y;
-                        *reinterpret_cast<float4 *>(dst + 4 * c) = o;
-                    }
+                    for (int c = 0; c < COLS / 4; ++c)
+                        atomicAdd(reinterpret_cast<float4 *>(dst + 4 * c),
+                                  make_float4(acc[2 * c].x, acc[2 * c].y, acc[2 * c + 1].x,
+                                              acc[2 * c + 1].y));
                 } else if (Cfg::TMA_STORE) {
                     // BF16 tile -> swizzled staging -> two bulk tensor stores per warp.
                     uint8_t *stg = sout + ew * Cfg::STAGE_OUT_WARP;
@@ -704,17 +703,48 @@ static cudaError_t run(const uint8_t *a, const float *sa, const uint8_t *b, cons
                        void *d, int64_t M, int64_t N, int64_t K, cudaStream_t stream, int num_sms)
 {
     auto kern = fp8_gemm_kernel<Cfg>;
-    cudaFuncAttributes attr;
-    cudaError_t e = cudaFuncGetAttributes(&attr, kern);
+    // Per-device launch facts, worked out on the first launch of this configuration on
+    // a device and cached: the register-split check, the shared-memory opt-in and (pair
+    // path) how many CTA pairs fit on the GPU at once.
+    static LaunchCache cache;
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
     if (e != cudaSuccess)
         return e;
-    // setmaxnreg.inc waits until enough registers are free; refuse to launch a
-    // split the launch allocation cannot cover (it would never make progress).
-    if (attr.numRegs * Cfg::THREADS < Cfg::REGS_NEEDED)
-        return cudaErrorInvalidConfiguration;
-    e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg::SMEM);
-    if (e != cudaSuccess)
-        return e;
+    int max_clusters = cache.get(dev);
+    if (max_clusters == 0) {
+        cudaFuncAttributes attr;
+        e = cudaFuncGetAttributes(&attr, kern);
+        if (e != cudaSuccess)
+            return e;
+        // setmaxnreg.inc waits until enough registers are free; refuse to launch a
+        // split the launch allocation cannot cover (it would never make progress).
+        if (attr.numRegs * Cfg::THREADS < Cfg::REGS_NEEDED)
+            return cudaErrorInvalidConfiguration;
+        e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg::SMEM);
+        if (e != cudaSuccess)
+            return e;
+        max_clusters = 1;
+        if (Cfg::CG == 2) {
+            cudaLaunchConfig_t q = {};
+            cudaLaunchAttribute qa[1];
+            qa[0].id = cudaLaunchAttributeClusterDimension;
+            qa[0].val.clusterDim.x = 2;
+            qa[0].val.clusterDim.y = 1;
+            qa[0].val.clusterDim.z = 1;
+            q.blockDim = dim3(Cfg::THREADS);
+            q.dynamicSmemBytes = Cfg::SMEM;
+            q.attrs = qa;
+            q.numAttrs = 1;
+            q.gridDim = dim3(2 * unsigned(num_sms / 2));
+            e = cudaOccupancyMaxActiveClusters(&max_clusters, kern, &q);
+            if (e != cudaSuccess)
+                return e;
+            if (max_clusters < 1)
+                return cudaErrorInvalidConfiguration;
+        }
+        cache.set(dev, max_clusters);
+    }
     CUtensorMap ta, tb;
     if (!make_map_u8(&ta, a, uint64_t(M), uint64_t(K), BM, BK))
         return cudaErrorInvalidValue;
@@ -751,13 +781,6 @@ static cudaError_t run(const uint8_t *a, const float *sa, const uint8_t *b, cons
     cfg.stream = stream;
     cfg.attrs = at;
     cfg.numAttrs = 1;
-    cfg.gridDim = dim3(2 * unsigned(num_sms / 2));
-    int max_clusters = 0;
-    e = cudaOccupancyMaxActiveClusters(&max_clusters, kern, &cfg);
-    if (e != cudaSuccess)
-        return e;
-    if (max_clusters < 1)
-        return cudaErrorInvalidConfiguration;
     const int64_t clusters = tiles < max_clusters ? tiles : max_clusters;
     cfg.gridDim = dim3(unsigned(2 * clusters));
     e = cudaLaunchKernelEx(&cfg, kern, ta, tb, td, sa, sb, dp, int(M), int(N), int(K));

@@ -37,6 +37,7 @@
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 
+#include "launch_cache.cuh"
 #include "ptx.cuh"
 #include "ptx_mx.cuh"
 #include "quant.cuh"
@@ -438,9 +439,40 @@ static cudaError_t run_mx(const uint8_t *a, const uint8_t *sa, const uint8_t *b,
                 CU_TENSOR_MAP_SWIZZLE_NONE))
         return cudaErrorInvalidValue;
     auto kern = fp8_gemm_mx_kernel<Cfg>;
-    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg::SMEM);
+    // Per-device launch facts, worked out on the first launch of this configuration on
+    // a device and cached: the shared-memory opt-in and (pair path) how many CTA pairs
+    // fit on the GPU at once.
+    static LaunchCache cache;
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
     if (e != cudaSuccess)
         return e;
+    int max_clusters = cache.get(dev);
+    if (max_clusters == 0) {
+        e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg::SMEM);
+        if (e != cudaSuccess)
+            return e;
+        max_clusters = 1;
+        if (Cfg::CG == 2) {
+            cudaLaunchConfig_t q = {};
+            cudaLaunchAttribute qa[1];
+            qa[0].id = cudaLaunchAttributeClusterDimension;
+            qa[0].val.clusterDim.x = 2;
+            qa[0].val.clusterDim.y = 1;
+            qa[0].val.clusterDim.z = 1;
+            q.blockDim = dim3(Cfg::THREADS);
+            q.dynamicSmemBytes = Cfg::SMEM;
+            q.attrs = qa;
+            q.numAttrs = 1;
+            q.gridDim = dim3(2 * unsigned(num_sms / 2));
+            e = cudaOccupancyMaxActiveClusters(&max_clusters, kern, &q);
+            if (e != cudaSuccess)
+                return e;
+            if (max_clusters < 1)
+                return cudaErrorInvalidConfiguration;
+        }
+        cache.set(dev, max_clusters);
+    }
     CUtensorMap ta, tb, td;
     const auto U8 = CU_TENSOR_MAP_DATA_TYPE_UINT8;
     if (!mx_map(&ta, U8, 1, a, uint64_t(M), uint64_t(K), MX_BM, MX_BK, CU_TENSOR_MAP_SWIZZLE_128B))
@@ -472,13 +504,6 @@ static cudaError_t run_mx(const uint8_t *a, const uint8_t *sa, const uint8_t *b,
     cfg.stream = stream;
     cfg.attrs = at;
     cfg.numAttrs = 1;
-    cfg.gridDim = dim3(2 * unsigned(num_sms / 2));
-    int max_clusters = 0;
-    e = cudaOccupancyMaxActiveClusters(&max_clusters, kern, &cfg);
-    if (e != cudaSuccess)
-        return e;
-    if (max_clusters < 1)
-        return cudaErrorInvalidConfiguration;
     const int64_t clusters = tiles < max_clusters ? tiles : max_clusters;
     cfg.gridDim = dim3(unsigned(2 * clusters));
     e = cudaLaunchKernelEx(&cfg, kern, ta, tb, td, tsa, tsb, int(M), int(N), int(K));

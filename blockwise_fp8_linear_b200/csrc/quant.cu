@@ -290,7 +290,11 @@ quant_tile_kernel(const __grid_constant__ CUtensorMap tmX, int64_t M, int64_t K,
         tma_load_2d(tile, &tmX, &bar, int32_t(kb * 128), int32_t(mb * 128));
     }
     __syncthreads();
-    if (!mbar_wait_bounded(&bar, 0u, &abort_flag, &g_quant_error, QERR_TILE_LOAD, QT_WAIT_NS)) {
+    const bool loaded =
+        mbar_wait_bounded(&bar, 0u, &abort_flag, &g_quant_error, QERR_TILE_LOAD, QT_WAIT_NS);
+    // Block-uniform decision: every thread leaves, or none does, so the barriers and
+    // full-warp shuffles below never run with exited threads.
+    if (__syncthreads_or(!loaded)) {
         if (t == 0) {  // keep the CTA (and its shared memory) alive while the copy may land
             const uint64_t t0 = global_timer_ns();
             while (global_timer_ns() - t0 < QT_DRAIN_NS) {

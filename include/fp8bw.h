@@ -14,10 +14,12 @@
  * fine-grained recipe section 3.2 says it follows, DeepSeek-V3).
  *
  * Conventions for every entry point
- *   Pointers     Device pointers on the calling thread's current CUDA device, unless
- *                stated otherwise.  The caller allocates and owns every buffer; the
- *                library never frees caller memory and keeps no pointer after the
- *                call returns.
+ *   Pointers     Device (or managed) pointers on the calling thread's current CUDA
+ *                device, unless stated otherwise; a host pointer or a buffer of
+ *                another device returns FP8BW_EINVAL before anything is launched.
+ *                The library never changes the current device.  The caller
+ *                allocates and owns every buffer; the library never frees caller
+ *                memory and keeps no pointer after the call returns.
  *   Layouts      Row-major [rows][cols].  BF16 tensors are IEEE bfloat16.  FP8 codes
  *                are E4M3 ("E4M3FN": bias 7, no infinities, NaN = S.1111.111).
  *                1x128 scale tensors are reduction-block-major, s[kb][row], so one

@@ -51,46 +51,69 @@ def test_single_process_defaults(monkeypatch):
     assert bench.max_over_ranks(3.5, 1) == 3.5
 
 
-def _rank_reduce(rank, world, port, out):
-    """Each rank makes its own dW per linear (seeded by rank), the reducer sums them over
-    the ranks and leaves rank r the rows [r*out/N, (r+1)*out/N)."""
+def _rank_reduce_fp32(rank, world, port, out):
+    """Each rank holds its own token shard of X and dY and computes the oracle's wgrad
+    over that shard as its local FP32 main gradient; the package's DpGradReducer sums
+    the FP32 gradients over the ranks (gloo reduce-scatter).  Rank r's rows must equal
+    the oracle's wgrad over the concatenated tokens within the FP32 rounding of the
+    exchange: each local gradient rounded once to binary32 plus one binary32 addition,
+    at most 3 * 2^-24 * sum_k |ahat_k bhat_k| per output."""
     import datetime
+    import numpy as np
     import torch
     import torch.distributed as dist
     os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
     dist.init_process_group("gloo", rank=rank, world_size=world,
                             timeout=datetime.timedelta(seconds=60))
-    import bench
-    shapes = [(256, 128), (512, 384)]
-    red = bench.DpGradReducer(shapes, world, "cpu")
+    import oracle
+    from blockwise_fp8_linear_b200 import synth
+    from blockwise_fp8_linear_b200.dp import DpGradReducer
 
-    def grad(r, i, dout, din):
-        g = torch.Generator().manual_seed(1000 * r + i)
-        # values on a coarse grid so that BF16 sums of two ranks are exact
-        return (torch.randint(-64, 64, (dout, din), generator=g).float() / 16).to(torch.bfloat16)
+    T, din, dout = 512, 256, 384                    # 256 tokens per rank: two 128-groups
+    X = synth.normal_bf16(T, din, 1.0, seed=synth.seed_for(77, 0), outliers=True)
+    dY = synth.normal_bf16(T, dout, 1e-3, seed=synth.seed_for(77, 2))
 
-    for i, (dout, din) in enumerate(shapes):
-        red.launch(i, grad(rank, i, dout, din))
+    def wgrad(x, dy):
+        a, sa = oracle.quant_act_t(np.ascontiguousarray(dy))
+        b, sb = oracle.quant_act_t(np.ascontiguousarray(x))
+        return oracle.gemm(oracle.WGRAD, a, sa, b, sb, dout, din, x.shape[0])
+
+    lo, hi = rank * T // world, (rank + 1) * T // world
+    local, _ = wgrad(X[lo:hi], dY[lo:hi])
+    red = DpGradReducer([(dout, din)], world, "cpu")
+    red.launch(0, torch.from_numpy(local.astype(np.float32)))
     red.wait()
-    ok = True
-    for i, (dout, din) in enumerate(shapes):
-        lo, hi = bench.DpGradReducer.rows(dout, world, rank)
-        want = sum(grad(r, i, dout, din).float() for r in range(world))[lo:hi]
-        ok = ok and torch.equal(red.shards[i].float(), want)
-    out[rank] = ok
+    full, asum = wgrad(X, dY)
+    r0, r1 = DpGradReducer.rows(dout, world, rank)
+    got = red.shards[0].double().numpy()
+    err = np.abs(got - full[r0:r1])
+    out[rank] = bool(np.all(err <= 3 * 2.0 ** -24 * asum[r0:r1])) and bool(np.any(got != 0))
     dist.destroy_process_group()
 
 
-def test_two_gloo_ranks_dw_reduce_scatter():
+def test_two_gloo_ranks_fp32_main_grad_reduce_scatter():
     world = 2
     port = _free_port()
     ctx = mp.get_context("spawn")
     mgr = ctx.Manager()
     out = mgr.dict()
-    procs = [ctx.Process(target=_rank_reduce, args=(r, world, port, out)) for r in range(world)]
+    procs = [ctx.Process(target=_rank_reduce_fp32, args=(r, world, port, out)) for r in range(world)]
     for p in procs:
         p.start()
     for p in procs:
-        p.join(120)
+        p.join(180)
         assert p.exitcode == 0
     assert dict(out) == {0: True, 1: True}
+
+
+def test_reducer_rejects_bad_shapes():
+    import torch
+    from blockwise_fp8_linear_b200.dp import DpGradReducer
+    import pytest
+    with pytest.raises(ValueError):
+        DpGradReducer([(130, 128)], 4, "cpu")
+    red = DpGradReducer([(256, 128)], 2, "cpu")
+    with pytest.raises(ValueError):
+        red.launch(0, torch.zeros(256, 128, dtype=torch.bfloat16))   # not the FP32 main grad
+    with pytest.raises(ValueError):
+        red.launch(0, torch.zeros(128, 256))

@@ -162,7 +162,10 @@ def test_gemm_e8m0_small_full(mode, T, Din, Dout):
     check_gemm(y, y_ref, asum, f"e8m0 mode {mode} {T}x{Din}x{Dout}")
 
 
-FULL = {"qkv": (8192, 2048, 4096), "gate_up": (8192, 2048, 12288), "down": (8192, 6144, 2048)}
+# gate: the MLP backward workload taken literally (one 6144-wide gate weight: dgrad
+# reduces over 6144, wgrad gives dW[6144][2048] over 8192 tokens)
+FULL = {"qkv": (8192, 2048, 4096), "gate_up": (8192, 2048, 12288), "down": (8192, 6144, 2048),
+        "gate": (8192, 2048, 6144)}
 
 
 @pytest.mark.parametrize("name", list(FULL))

@@ -127,6 +127,22 @@ def test_gemm_full_size_sampled(name, mode):
     check_gemm(y, y_ref, asum, f"{name} mode {mode}")
 
 
+# The MLP backward workload taken literally: one 6144-wide gate (or up) weight, so
+# dgrad reduces over 6144 into dX[8192][2048] and wgrad gives dW[6144][2048] over 8192
+# tokens (the down projection's dgrad and wgrad are the "down" rows above).
+MLP_BWD = {"gate": (8192, 2048, 6144)}
+
+
+@pytest.mark.parametrize("mode", [FPROP, DGRAD, WGRAD])
+def test_gemm_mlp_backward_shapes_sampled(mode):
+    T, Din, Dout = MLP_BWD["gate"]
+    X, W, dY = _layer(T, Din, Dout, seed=613 + mode)
+    M = {FPROP: T, DGRAD: T, WGRAD: Dout}[mode]
+    rows = _rows(M, 24)
+    y, y_ref, asum = _run_mode(mode, X, W, dY, rows=rows)
+    check_gemm(y, y_ref, asum, f"gate 6144 mode {mode}")
+
+
 # The micro-batch sweep of a 28-layer step runs the same four linears at M = 4096, 16384
 # and 32768 tokens (micro-batch 1, 4, 8 x sequence 4096): every linear at the smallest,
 # one linear at each of the larger sizes (the wgrad reduction grows to 32768 tokens).
@@ -200,3 +216,35 @@ def test_wgrad_fp32_accumulation(T, Din, Dout):
     check_gemm(y1, p64 + y_ref, asum + np.abs(p64), "acc32 once")
     check_gemm(y2, p64 + 2 * y_ref, 2 * asum + np.abs(p64), "acc32 twice")
 
+
+
+@pytest.mark.parametrize("T,Din,Dout", [
+    (256, 384, 640),      # single-CTA path (vector atomic adds)
+    (8192, 2048, 4096),   # CTA-pair path (TMA reduce-add), rows sampled
+])
+def test_wgrad_fp32_accumulation_overlapping_calls(T, Din, Dout):
+    """Two fp8_gemm_wgrad_acc32 calls on two streams, free to overlap on the GPU, into
+    one FP32 buffer: both sums must land (prev + 2 * sum), only their order may vary."""
+    X, W, dY = _layer(T, Din, Dout, seed=T + Din + Dout + 57)
+    a_d, sa_d = fp8_quant_act_t(to_dev_bf16(dY))
+    b_d, sb_d = fp8_quant_act_t(to_dev_bf16(X))
+    a, sa = oracle.quant_act_t(dY)
+    b, sb = oracle.quant_act_t(X)
+    M, N, K = Dout, Din, T
+    rows = _rows(M, 24) if M * N > 4 * 1024 * 1024 else None
+    rng = np.random.default_rng(11)
+    prev = (rng.standard_normal((M, N)) * 1e-3).astype(np.float32)
+    dw = torch.from_numpy(prev.copy()).cuda()
+    s1, s2 = torch.cuda.Stream(), torch.cuda.Stream()
+    start = torch.cuda.Event()
+    start.record()
+    for st in (s1, s2):
+        st.wait_event(start)
+        fp8_gemm_wgrad_acc32(a_d, sa_d, b_d, sb_d, M, N, K, dw, stream=st)
+    torch.cuda.synchronize()
+    y2 = dw.cpu().numpy().astype(np.float64)
+    y_ref, asum = oracle.gemm(WGRAD, a, sa, b, sb, M, N, K, rows=rows)
+    p64 = prev.astype(np.float64)
+    if rows is not None:
+        y2, p64 = y2[rows], p64[rows]
+    check_gemm(y2, p64 + 2 * y_ref, 2 * asum + np.abs(p64), "acc32 on two streams")
