@@ -803,16 +803,18 @@ KERNEL_CASES = ("gemm_fprop", "gemm_dgrad", "gemm_wgrad", "gemm_mx_fprop", "gemm
 
 
 def run_kernel_only(args):
-    """Launch one kernel of the step (QKV linear shapes: M=8192, 2048 -> 4096; the
-    quantizers on the 8192x12288 gate/up gradient so inputs exceed L2) warmup+steps
-    times back to back and print its mean device time.  For profilers."""
+    """Launch one kernel of the step (the GEMMs on one linear's shapes, --kernel-linear,
+    QKV by default: M=8192, 2048 -> 4096; the quantizers on the 8192x12288 gate/up
+    gradient so inputs exceed L2) warmup+steps times back to back and print its mean
+    device time.  For profilers."""
     import torch
     import blockwise_fp8_linear_b200 as fb
     from blockwise_fp8_linear_b200 import build as fbuild
     fbuild.build()
     dev = torch.device("cuda", 0)
     g = torch.Generator(device=dev).manual_seed(0)
-    T, din, dout = TOKENS, 2048, 4096
+    T = TOKENS
+    _, din, dout = next(x for x in LINEARS if x[0] == args.kernel_linear)
     case = args.kernel_only
 
     def randn(r, c, std):
@@ -873,7 +875,7 @@ def run_kernel_only(args):
     e1.record()
     torch.cuda.synchronize()
     ms = e0.elapsed_time(e1) / args.steps
-    print(json.dumps({"kernel_only": case, "ms": round(ms, 5),
+    print(json.dumps({"kernel_only": case, "linear": args.kernel_linear, "ms": round(ms, 5),
                       work[0]: round(work[1] / (ms * 1e-3), 2)}), flush=True)
 
 
@@ -1016,6 +1018,8 @@ def main():
                     help="run every kernel on one stream (no dgrad/wgrad overlap)")
     ap.add_argument("--kernel-only", choices=KERNEL_CASES, default=None,
                     help="launch one kernel repeatedly (for profilers); no JSON metric line")
+    ap.add_argument("--kernel-linear", choices=[n for n, _, _ in LINEARS], default="qkv",
+                    help="with --kernel-only gemm_*: the linear whose GEMM shapes to launch")
     ap.add_argument("--sweep", action="store_true",
                     help="micro-batch knee sweep (28 layers, M = 4096..32768); one JSON line per M")
     ap.add_argument("--sweep-steps", type=int, default=3)

@@ -158,6 +158,8 @@ fp8_gemm_mx_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constan
     else
         __syncthreads();
     tc_fence_after();
+    pdl_wait();               // inputs written by the previous kernel are visible
+    pdl_launch_dependents();  // the next kernel may start its launch and prologue
     const uint32_t tmem_base = *tmem_slot;
     const uint32_t full_lead = (CG == 2) ? mapa_shared(smem_u32(full), 0) : smem_u32(full);
     const uint32_t tempty_lead = (CG == 2) ? mapa_shared(smem_u32(tempty), 0) : smem_u32(tempty);
@@ -488,24 +490,25 @@ static cudaError_t run_mx(const uint8_t *a, const uint8_t *sa, const uint8_t *b,
                 CU_TENSOR_MAP_SWIZZLE_128B))
         return cudaErrorInvalidValue;
     const int64_t tiles = (M / Cfg::TILE_M) * (N / Cfg::BN);
-    if (Cfg::CG == 1) {
-        const int grid = int(tiles < num_sms ? tiles : num_sms);
-        kern<<<grid, Cfg::THREADS, Cfg::SMEM, stream>>>(ta, tb, td, tsa, tsb, int(M), int(N), int(K));
-        return cudaGetLastError();
-    }
     cudaLaunchConfig_t cfg = {};
-    cudaLaunchAttribute at[1];
-    at[0].id = cudaLaunchAttributeClusterDimension;
-    at[0].val.clusterDim.x = 2;
-    at[0].val.clusterDim.y = 1;
-    at[0].val.clusterDim.z = 1;
+    cudaLaunchAttribute at[2];
+    set_pdl(at[0]);
+    at[1].id = cudaLaunchAttributeClusterDimension;
+    at[1].val.clusterDim.x = 2;
+    at[1].val.clusterDim.y = 1;
+    at[1].val.clusterDim.z = 1;
     cfg.blockDim = dim3(Cfg::THREADS);
     cfg.dynamicSmemBytes = Cfg::SMEM;
     cfg.stream = stream;
     cfg.attrs = at;
-    cfg.numAttrs = 1;
-    const int64_t clusters = tiles < max_clusters ? tiles : max_clusters;
-    cfg.gridDim = dim3(unsigned(2 * clusters));
+    if (Cfg::CG == 1) {
+        cfg.numAttrs = 1;
+        cfg.gridDim = dim3(unsigned(tiles < num_sms ? tiles : num_sms));
+    } else {
+        cfg.numAttrs = 2;
+        const int64_t clusters = tiles < max_clusters ? tiles : max_clusters;
+        cfg.gridDim = dim3(unsigned(2 * clusters));
+    }
     e = cudaLaunchKernelEx(&cfg, kern, ta, tb, td, tsa, tsb, int(M), int(N), int(K));
     if (e != cudaSuccess)
         return e;

@@ -5,6 +5,7 @@
 #pragma once
 
 #include <atomic>
+#include <cuda_runtime.h>
 
 namespace fp8bw {
 
@@ -24,5 +25,18 @@ struct LaunchCache {
             clusters[dev].store(v, std::memory_order_release);
     }
 };
+
+#ifndef FP8BW_PDL
+#define FP8BW_PDL 1
+#endif
+// Programmatic stream serialization: the kernel may be launched while the previous
+// kernel in the stream is still finishing (every kernel of this library waits for
+// its predecessor with griddepcontrol.wait before touching memory), so launch
+// latency and prologue (barrier set-up, tensor-memory allocation) overlap that tail.
+inline void set_pdl(cudaLaunchAttribute &a)
+{
+    a.id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    a.val.programmaticStreamSerializationAllowed = FP8BW_PDL;
+}
 
 } // namespace fp8bw

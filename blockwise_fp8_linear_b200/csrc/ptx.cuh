@@ -38,6 +38,23 @@ __device__ __forceinline__ void regs_inc()
     asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(N));
 }
 
+// ------------------------------------------------ programmatic dependent launch
+
+// Wait until the kernels this grid depends on (the previous kernel in the stream,
+// when this one was launched with programmatic stream serialization) have completed
+// and their memory writes are visible.  Called before any global-memory access.
+__device__ __forceinline__ void pdl_wait()
+{
+    asm volatile("griddepcontrol.wait;" ::: "memory");
+}
+
+// Allow the next kernel in the stream to start launching; its CTAs still call
+// pdl_wait() before they touch memory, so this only overlaps launch and prologue.
+__device__ __forceinline__ void pdl_launch_dependents()
+{
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
 // ------------------------------------------------------------------ mbarrier
 
 __device__ __forceinline__ void mbar_init(uint64_t *bar, uint32_t count)

@@ -14,6 +14,7 @@
 #include <cuda.h>
 #include <cuda_runtime.h>
 
+#include "launch_cache.cuh"
 #include "ptx.cuh"
 #include "quant.cuh"
 
@@ -173,6 +174,8 @@ quant_weight_kernel(const uint4 *__restrict__ w, int64_t N, int64_t K, uint2 *__
     const int t = threadIdx.x;
     const int64_t kb = blockIdx.x, nb = blockIdx.y;
     const int rsub = t >> 4, csub = (t & 15) * 8;
+    pdl_wait();
+    pdl_launch_dependents();
 
     uint4 v[8];
 #pragma unroll
@@ -282,6 +285,8 @@ quant_tile_kernel(const __grid_constant__ CUtensorMap tmX, int64_t M, int64_t K,
     const int64_t kb = blockIdx.x, mb = blockIdx.y;
     const int rsub = t >> 4, sub = t & 15;
 
+    pdl_wait();               // X (and the output buffers) are free of the previous kernel
+    pdl_launch_dependents();
     if (t == 0) {
         mbar_init(&bar, 1);
         abort_flag = 0;
@@ -486,10 +491,17 @@ static cudaError_t run_tile(const void *x, int64_t M, int64_t K, void *q, void *
     CUtensorMap map;
     if (!tile_map_bf16(&map, x, M, K))
         return cudaErrorInvalidValue;
-    dim3 grid(unsigned(K / 128), unsigned(M / 128));
-    quant_tile_kernel<ROWS, COLS, E8><<<grid, QD_THREADS, 0, stream>>>(
-        map, M, K, reinterpret_cast<uint2 *>(q), s, qt, st);
-    return cudaGetLastError();
+    cudaLaunchConfig_t cfg = {};
+    cudaLaunchAttribute at[1];
+    set_pdl(at[0]);
+    cfg.gridDim = dim3(unsigned(K / 128), unsigned(M / 128));
+    cfg.blockDim = dim3(QD_THREADS);
+    cfg.stream = stream;
+    cfg.attrs = at;
+    cfg.numAttrs = 1;
+    cudaError_t e = cudaLaunchKernelEx(&cfg, quant_tile_kernel<ROWS, COLS, E8>, map, M, K,
+                                       reinterpret_cast<uint2 *>(q), s, qt, st);
+    return e != cudaSuccess ? e : cudaGetLastError();
 }
 
 cudaError_t read_and_clear_quant_error(int *value)
@@ -502,6 +514,23 @@ cudaError_t read_and_clear_quant_error(int *value)
         e = cudaMemcpyToSymbol(g_quant_error, &zero, sizeof(int));
     }
     return e;
+}
+
+template <bool E8>
+static cudaError_t run_weight(const void *w, int64_t N, int64_t K, void *q, void *s, uint8_t *qt,
+                              cudaStream_t stream)
+{
+    cudaLaunchConfig_t cfg = {};
+    cudaLaunchAttribute at[1];
+    set_pdl(at[0]);
+    cfg.gridDim = dim3(unsigned(K / 128), unsigned(N / 128));
+    cfg.blockDim = dim3(QW_THREADS);
+    cfg.stream = stream;
+    cfg.attrs = at;
+    cfg.numAttrs = 1;
+    cudaError_t e = cudaLaunchKernelEx(&cfg, quant_weight_kernel<E8>, static_cast<const uint4 *>(w),
+                                       N, K, reinterpret_cast<uint2 *>(q), s, qt);
+    return e != cudaSuccess ? e : cudaGetLastError();
 }
 
 // ------------------------------------------------------------------ launchers
@@ -527,10 +556,7 @@ cudaError_t launch_quant_act_t(const void *x, int64_t M, int64_t K, uint8_t *qt,
 cudaError_t launch_quant_weight(const void *w, int64_t N, int64_t K, uint8_t *q, float *s,
                                 uint8_t *qt, cudaStream_t stream)
 {
-    dim3 grid(unsigned(K / 128), unsigned(N / 128));
-    quant_weight_kernel<false><<<grid, QW_THREADS, 0, stream>>>(
-        static_cast<const uint4 *>(w), N, K, reinterpret_cast<uint2 *>(q), s, qt);
-    return cudaGetLastError();
+    return run_weight<false>(w, N, K, q, s, qt, stream);
 }
 
 // Power-of-two (E8M0) scale quantizers: the same code layouts, scales as 512-byte
@@ -546,10 +572,7 @@ cudaError_t launch_quant_e8m0(int which, const void *x, int64_t M, int64_t K, ui
     case 2:  // both
         return run_tile<true, true, true>(x, M, K, q, s, qt, st, stream);
     default: {  // weight blocks: q[N=M][K], s[M/128][K/128], optional qt[K][M]
-        dim3 grid(unsigned(K / 128), unsigned(M / 128));
-        quant_weight_kernel<true><<<grid, QW_THREADS, 0, stream>>>(
-            static_cast<const uint4 *>(x), M, K, reinterpret_cast<uint2 *>(q), s, qt);
-        return cudaGetLastError();
+        return run_weight<true>(x, M, K, q, s, qt, stream);
     }
     }
 }

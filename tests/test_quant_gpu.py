@@ -24,7 +24,9 @@ def _eq_bits(gpu: torch.Tensor, ref: np.ndarray, what: str):
         raise AssertionError(f"{what}: {len(bad)} mismatches, first at {i}: gpu={g[i]:#x} ref={ref[i]:#x}")
 
 
-ACT_SHAPES = [(128, 1024), (384, 640), (256, 128), (8192, 2048), (8192, 6144), (32768, 2048)]
+# (16384, 2048): the activation shape of a 16k-token batch at model width 2048
+ACT_SHAPES = [(128, 1024), (384, 640), (256, 128), (8192, 2048), (16384, 2048), (8192, 6144),
+              (32768, 2048)]
 
 
 @pytest.mark.parametrize("M,K", ACT_SHAPES)
