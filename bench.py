@@ -372,6 +372,21 @@ def gemm_summary(gemm_events, work):
              "tflops": round(ff / (t * 1e-3) / 1e12, 1)} for k, (t, ff, n) in acc.items()]
 
 
+def quant_kernel_rows(dev, quant_rows, hbm_peak, steps):
+    rows = []
+    for r in quant_rows:
+        shape = tuple(r["shape"])
+        per_elem = DUAL_BYTES if r["kernel"] == "quant_act_dual" else WEIGHT_BYTES
+        us = quant_stream_us(dev, r["kernel"], shape)
+        gbs = shape[0] * shape[1] * per_elem / (us * 1e-6) / 1e9
+        rows.append({"kernel": r["kernel"], "shape": list(shape), "launches_per_step":
+                     r["launches"] // max(1, steps), "us": round(us, 2),
+                     "gbs": round(gbs, 1), "frac": round(gbs / hbm_peak, 4),
+                     "frac_of_nominal": round(gbs / NOMINAL_HBM_GBS, 4),
+                     "in_step_us": r["us"]})
+    return rows
+
+
 def quant_summary(quant_events):
     """GB/s of each quantizer kind and shape (algorithmic bytes / mean device time)."""
     acc = {}
@@ -381,6 +396,58 @@ def quant_summary(quant_events):
         acc[key] = (t + e0.elapsed_time(e1), b + nbytes, n + 1)
     return [{"kernel": k, "shape": list(shp), "launches": n, "us": round(1e3 * t / n, 2),
              "gbs": round(b / (t * 1e-3) / 1e9, 1)} for (k, shp), (t, b, n) in sorted(acc.items())]
+
+
+L2_BYTES = 126 * 2 ** 20  # B200 L2
+
+
+def quant_stream_us(dev, kind, shape):
+    """Device time per launch of one quantizer kind and shape, launched back to back
+    through the C ABI as in the step (programmatic dependent launch lets each launch's
+    prologue overlap the previous one's tail).  Inputs and outputs rotate over enough
+    copies to exceed twice the L2, so every launch reads its BF16 input from HBM; the
+    event-bracketed in-step time also carries the launch gap that the brackets force."""
+    import torch
+    import blockwise_fp8_linear_b200 as fb
+    L = fb.lib()
+    st = torch.cuda.current_stream().cuda_stream
+    R, C = shape
+    n = max(2, -(-2 * L2_BYTES // (R * C * 2)))
+    g = torch.Generator(device=dev).manual_seed(1)
+    u8 = lambda r, c: torch.empty(r, c, dtype=torch.uint8, device=dev)
+    f32 = lambda r, c: torch.empty(r, c, dtype=torch.float32, device=dev)
+    bufs = []
+    for _ in range(n):
+        x = torch.randn(R, C, device=dev, generator=g).to(torch.bfloat16)
+        if kind == "quant_act_dual":
+            bufs.append((x, u8(R, C), f32(C // 128, R), u8(C, R), f32(R // 128, C)))
+        else:
+            bufs.append((x, u8(R, C), f32(R // 128, C // 128)))
+
+    def launch(i):
+        b = [t.data_ptr() for t in bufs[i]]
+        if kind == "quant_act_dual":
+            rc = L.fp8_quant_act_dual(b[0], R, C, b[1], b[2], b[3], b[4], st)
+        else:
+            rc = L.fp8_quant_weight(b[0], R, C, b[1], b[2], None, st)
+        if rc:
+            raise fb.Fp8bwError(rc, kind)
+
+    for i in range(n):
+        launch(i)
+    reps = max(4 * n, 40)
+    torch.cuda.synchronize()
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for k in range(reps):
+        launch(k % n)
+    e1.record()
+    torch.cuda.synchronize()
+    us = e0.elapsed_time(e1) * 1e3 / reps
+    del bufs
+    torch.cuda.empty_cache()
+    return us
 
 
 def single_fprop_latency(dev, reps=200):
@@ -632,10 +699,12 @@ def run_ours(args):
         "target": ">= 0.75 of HBM bandwidth, reported against both the measured copy "
                   "bandwidth (frac) and the nominal 8 TB/s (frac_of_nominal)",
         "bytes_per_element": {"quant_act_dual": DUAL_BYTES, "quant_weight": WEIGHT_BYTES},
-        "measured_on": "the same one-stream pass, every quantizer launch bracketed by events",
-        "kernels": [dict(r, frac=round(r["gbs"] / hbm_peak, 4),
-                         frac_of_nominal=round(r["gbs"] / NOMINAL_HBM_GBS, 4))
-                    for r in quant_rows],
+        "measured_on": "us / gbs / frac: each kind and shape launched back to back through the "
+                       "C ABI, inputs and outputs rotating over copies larger than twice the "
+                       "L2 (every launch reads HBM); in_step_us: the same launches inside the "
+                       "one-stream pass, each bracketed by events (adds the launch gap the "
+                       "brackets force)",
+        "kernels": quant_kernel_rows(dev, quant_rows, hbm_peak, args.steps),
     }
     single = single_fprop_latency(dev) if not args.no_single else None
 
@@ -804,9 +873,9 @@ KERNEL_CASES = ("gemm_fprop", "gemm_dgrad", "gemm_wgrad", "gemm_mx_fprop", "gemm
 
 def run_kernel_only(args):
     """Launch one kernel of the step (the GEMMs on one linear's shapes, --kernel-linear,
-    QKV by default: M=8192, 2048 -> 4096; the quantizers on the 8192x12288 gate/up
-    gradient so inputs exceed L2) warmup+steps times back to back and print its mean
-    device time.  For profilers."""
+    QKV by default: M=8192, 2048 -> 4096; the quantizers on --quant-shape, by default
+    the 8192x12288 gate/up gradient so inputs exceed L2) warmup+steps times back to back
+    and print its mean device time.  For profilers."""
     import torch
     import blockwise_fp8_linear_b200 as fb
     from blockwise_fp8_linear_b200 import build as fbuild
@@ -849,18 +918,36 @@ def run_kernel_only(args):
             flops = 2 * T * din * dout
         work = ("TFLOP/s", flops / 1e12)
     else:
-        R, C = T, 12288
+        R, C = (int(v) for v in args.quant_shape.split("x"))
         X = randn(R, C, 1.0)
-        if case == "quant_act":
-            launch = lambda: fb.fp8_quant_act(X)
-        elif case == "quant_act_t":
-            launch = lambda: fb.fp8_quant_act_t(X)
-        elif case == "quant_dual":
-            launch = lambda: fb.fp8_quant_act_dual(X)
-        elif case == "quant_dual_e8m0":
-            launch = lambda: fb.fp8_quant_act_dual_e8m0(X)
+        # outputs allocated once and the C ABI called directly, so that host work per
+        # launch stays well below the kernel time even for the small shapes
+        L = fb.lib()
+        st = fb._stream(None)
+        u8 = lambda r, c: torch.empty(r, c, dtype=torch.uint8, device=dev)
+        f32 = lambda r, c: torch.empty(r, c, dtype=torch.float32, device=dev)
+        q, qt = u8(R, C), u8(C, R)
+        if case == "quant_dual_e8m0":
+            s, sT = u8(R // 128, (C // 128) * 512), u8(C // 128, (R // 128) * 512)
         else:
-            launch = lambda: fb.fp8_quant_weight(X)
+            s, sT = f32(C // 128, R), f32(R // 128, C)
+        p = lambda x: x.data_ptr()
+
+        def run(fn, *a):
+            rc = fn(*a)
+            if rc:
+                raise fb.Fp8bwError(rc, case)
+        if case == "quant_act":
+            launch = lambda: run(L.fp8_quant_act, p(X), R, C, p(q), p(s), st)
+        elif case == "quant_act_t":
+            launch = lambda: run(L.fp8_quant_act_t, p(X), R, C, p(qt), p(sT), st)
+        elif case == "quant_dual":
+            launch = lambda: run(L.fp8_quant_act_dual, p(X), R, C, p(q), p(s), p(qt), p(sT), st)
+        elif case == "quant_dual_e8m0":
+            launch = lambda: run(L.fp8_quant_act_dual_e8m0, p(X), R, C, p(q), p(s), p(qt), p(sT), st)
+        else:
+            sw = f32(R // 128, C // 128)
+            launch = lambda: run(L.fp8_quant_weight, p(X), R, C, p(q), p(sw), None, st)
         per_elem = (4 + 8 / 128) if case.startswith("quant_dual") else (3 + 4 / 128)
         work = ("GB/s", R * C * per_elem / 1e9)
     torch.cuda.synchronize()
@@ -875,7 +962,8 @@ def run_kernel_only(args):
     e1.record()
     torch.cuda.synchronize()
     ms = e0.elapsed_time(e1) / args.steps
-    print(json.dumps({"kernel_only": case, "linear": args.kernel_linear, "ms": round(ms, 5),
+    print(json.dumps({"kernel_only": case, "linear": args.kernel_linear,
+                      "quant_shape": args.quant_shape, "ms": round(ms, 5),
                       work[0]: round(work[1] / (ms * 1e-3), 2)}), flush=True)
 
 
@@ -1020,6 +1108,8 @@ def main():
                     help="launch one kernel repeatedly (for profilers); no JSON metric line")
     ap.add_argument("--kernel-linear", choices=[n for n, _, _ in LINEARS], default="qkv",
                     help="with --kernel-only gemm_*: the linear whose GEMM shapes to launch")
+    ap.add_argument("--quant-shape", default="8192x12288",
+                    help="with --kernel-only quant_*: ROWSxCOLS of the BF16 input")
     ap.add_argument("--sweep", action="store_true",
                     help="micro-batch knee sweep (28 layers, M = 4096..32768); one JSON line per M")
     ap.add_argument("--sweep-steps", type=int, default=3)
