@@ -804,7 +804,10 @@ cudaError_t launch_gemm(int mode, const uint8_t *a, const float *sa, const uint8
 {
     constexpr int PBN = FP8BW_PAIR_BN;                 // N of a pair tile
     constexpr int PST = (PBN == 256) ? 4 : 6;          // pair-path pipeline stages
-    const bool wide = (N % 256) == 0;
+    // Single-CTA path: 128-wide tiles when N is not a multiple of 256, and also when
+    // 256-wide ones would leave most SMs idle (fewer tiles than half the SMs, e.g. the
+    // 128 x 1024 x 1024 single-layer fprop: 4 tiles of 128 x 256 or 8 of 128 x 128).
+    const bool wide = (N % 256) == 0 && (M / 128) * (N / 256) * 2 >= num_sms;
     const bool pair = FP8BW_PAIR && (N % PBN) == 0 && (M % 256) == 0 &&
                       (M / 256) * (N / PBN) >= 16;
     switch (mode) {

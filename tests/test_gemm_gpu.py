@@ -86,6 +86,16 @@ def test_gemm_small_full(mode, T, Din, Dout):
     check_gemm(y, y_ref, asum, f"mode {mode} {T}x{Din}x{Dout}")
 
 
+@pytest.mark.parametrize("mode,T,Din,Dout", [
+    (FPROP, 384, 256, 6400), (DGRAD, 384, 6400, 256), (WGRAD, 256, 6400, 384)])
+def test_gemm_single_cta_wide_tiles(mode, T, Din, Dout):
+    """M = 384 (not a multiple of 256), N = 6400, K = 256: the single-CTA path with
+    128 x 256 tiles (75 of them, enough to keep that width); every output checked."""
+    X, W, dY = _layer(T, Din, Dout, seed=4242 + mode)
+    y, y_ref, asum = _run_mode(mode, X, W, dY)
+    check_gemm(y, y_ref, asum, f"mode {mode} single-CTA 128x256 tiles")
+
+
 def test_gemm_single_fprop_workload():
     """X[128x1024] ~ N(0,1), W[1024x1024] ~ N(0,0.02), seed 0: Y = X W^T, checked
     on every output."""
