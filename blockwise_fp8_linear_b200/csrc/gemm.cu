@@ -329,6 +329,17 @@ fp8_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__
                     } else if (MODE == 1) {
                         if (lane < BN / 128)
                             cp_async_4(slot + BM + lane, sb + size_t(kb) * (N / 128) + nb0 + lane);
+                    } else if (Cfg::WG16) {
+                        // Column scales in the order the 16x256b promotion reads them:
+                        // column 128 h + 64 cc + 8 j + 2 t0 + e goes to slot position
+                        // 128 h + 64 cc + 16 t0 + 2 j + e, so a thread's 16 scales of one
+                        // 64-column chunk are contiguous (four 16-byte loads).  Lane l copies
+                        // columns 8 l .. 8 l + 7 (j = l % 8) as four 8-byte pieces.
+                        const float *src = sb + size_t(kb) * N + tn * BN + lane * 8;
+                        float *dst = slot + BM + (lane >> 3) * 64 + (lane & 7) * 2;
+#pragma unroll
+                        for (int q = 0; q < 4; ++q)
+                            cp_async_8(dst + 16 * q, src + 2 * q);
                     } else {
                         const float *src = sb + size_t(kb) * N + tn * BN + lane * (BN / 32);
 #pragma unroll
@@ -396,10 +407,18 @@ fp8_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__
 #pragma unroll
                 for (int cc = 0; cc < 2; ++cc) {
                     float2 sbp[8];
+                    {
+                        // this thread's 16 column scales of chunk cc, contiguous (see the
+                        // scale loader)
+                        const float4 *sp =
+                            reinterpret_cast<const float4 *>(slot + BM + col0 + 64 * cc + 16 * t0);
 #pragma unroll
-                    for (int j = 0; j < 8; ++j)
-                        sbp[j] = *reinterpret_cast<const float2 *>(slot + BM + col0 + 64 * cc +
-                                                                   8 * j + 2 * t0);
+                        for (int m = 0; m < 4; ++m) {
+                            const float4 v = sp[m];
+                            sbp[2 * m] = make_float2(v.x, v.y);
+                            sbp[2 * m + 1] = make_float2(v.z, v.w);
+                        }
+                    }
 #pragma unroll
                     for (int h = 0; h < 2; ++h) {
                         uint32_t v[32];
