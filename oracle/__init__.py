@@ -105,7 +105,7 @@ def quantize_group(x_bf16: np.ndarray):
 
 
 def quant_act(x_bf16: np.ndarray):
-    """X[M][K] -> (Q[M][K] uint8, S[K/128][M] float32)."""
+    """X[M][K] -> (Q[M][K] uint8, S[K/128][M] float32); any token count M."""
     x = _u16(x_bf16)
     M, K = x.shape
     q = np.empty((M, K), dtype=np.uint8)
@@ -117,11 +117,12 @@ def quant_act(x_bf16: np.ndarray):
 
 
 def quant_act_t(x_bf16: np.ndarray):
-    """X[M][K] -> (Q^T[K][M] uint8, S^T[M/128][K] float32)."""
+    """X[M][K] -> (Q^T[K][M] uint8, S^T[ceil(M/128)][K] float32).  M may be any token
+    count: the last token group holds M mod 128 tokens, its scale taken over them."""
     x = _u16(x_bf16)
     M, K = x.shape
     qt = np.empty((K, M), dtype=np.uint8)
-    st = np.empty((M // 128, K), dtype=np.float32)
+    st = np.empty(((M + 127) // 128, K), dtype=np.float32)
     rc = _load().fp8o_quant_act_t(_ptr(x), M, K, _ptr(qt), _ptr(st))
     if rc:
         raise ValueError(f"oracle quant_act_t: bad sizes {M}x{K}")

@@ -14,7 +14,11 @@
  *     and the FP32 quotient is rounded to E4M3 with ties-to-even, saturating at
  *     +-448: two roundings by definition;
  *   - an all-zero group gets scale 0 and codes 0x00, with no division;
- *   - in a nonzero group the sign of a zero or underflowing value is kept.
+ *   - in a nonzero group the sign of a zero or underflowing value is kept;
+ *   - a token count that is not a multiple of 128 leaves a last group of M mod 128
+ *     tokens along the token dimension: its amax, and so its scale, is taken over
+ *     the tokens present, and codes exist only for them (the same result as
+ *     zero-padding the tokens to a multiple of 128, since zeros change no amax).
  *
  * Compile with IEEE binary32 arithmetic (x86-64 SSE, -ffp-contract=off, no
  * fast-math) so that the two divisions round exactly once each.
@@ -127,9 +131,15 @@ static int bad_sizes(int64_t a, int64_t b)
     return a <= 0 || b <= 0 || (a % 128) != 0 || (b % 128) != 0;
 }
 
+/* Activations: any token count M > 0, features K a multiple of 128. */
+static int bad_act_sizes(int64_t M, int64_t K)
+{
+    return M <= 0 || K <= 0 || (K % 128) != 0;
+}
+
 int fp8o_quant_act(const uint16_t *x, int64_t M, int64_t K, uint8_t *q, float *s)
 {
-    if (bad_sizes(M, K))
+    if (bad_act_sizes(M, K))
         return -1;
     int64_t KB = K / 128;
 #pragma omp parallel for schedule(static)
@@ -142,14 +152,16 @@ int fp8o_quant_act(const uint16_t *x, int64_t M, int64_t K, uint8_t *q, float *s
 
 int fp8o_quant_act_t(const uint16_t *x, int64_t M, int64_t K, uint8_t *qt, float *st)
 {
-    if (bad_sizes(M, K))
+    if (bad_act_sizes(M, K))
         return -1;
-    int64_t MB = M / 128;
+    int64_t MB = (M + 127) / 128; /* the last group may hold fewer than 128 tokens */
 #pragma omp parallel for schedule(static)
     for (int64_t k = 0; k < K; ++k)
-        for (int64_t mb = 0; mb < MB; ++mb)
-            st[mb * K + k] = fp8o_quantize_group(x + mb * 128 * K + k, K, 128,
+        for (int64_t mb = 0; mb < MB; ++mb) {
+            int64_t n = M - mb * 128 < 128 ? M - mb * 128 : 128;
+            st[mb * K + k] = fp8o_quantize_group(x + mb * 128 * K + k, K, n,
                                                  qt + k * M + mb * 128, 1);
+        }
     return 0;
 }
 
@@ -334,8 +346,12 @@ int fp8o_gemm(int mode, const uint8_t *a, const float *sa, const uint8_t *b,
               const int64_t *rows, int64_t nrows, double *y, double *asum,
               int nthreads)
 {
-    if (mode < 0 || mode > 2 || M <= 0 || N <= 0 || K <= 0 ||
-        (M % 128) || (N % 128) || (K % 128))
+    /* Tokens may be any count: M for FPROP/DGRAD (a[M][K], sa[K/128][M]), the
+     * reduction K for WGRAD (a[M][K], sa[ceil(K/128)][M], sb[ceil(K/128)][N]; the
+     * last block holds K mod 128 tokens).  Feature dimensions are multiples of 128. */
+    if (mode < 0 || mode > 2 || M <= 0 || N <= 0 || K <= 0 || (N % 128))
+        return -1;
+    if (mode == 2 ? (M % 128) != 0 : (K % 128) != 0)
         return -1;
     if (!rows)
         nrows = M;

@@ -166,3 +166,63 @@ def test_bad_arguments_rejected():
         oracle.gemm(3, z, s, z, s, 128, 128, 128)
     with pytest.raises(ValueError):
         oracle.gemm(0, z, s, z, s, 128, 128, 100)
+
+
+# ---- token counts that are not a multiple of 128 ----
+
+def _dequant_a_ragged(a, sa, K):
+    """ahat[m][k] = code * sa[k/128][m] for a reduction K that may end in a partial block."""
+    return VALS[a] * np.repeat(sa.astype(np.float64), 128, axis=0)[:K].T
+
+
+@pytest.mark.parametrize("mode,M", [(0, 200), (1, 16), (0, 144)])
+def test_gemm_ragged_tokens_fprop_dgrad(mode, M):
+    """FPROP / DGRAD with M tokens not a multiple of 128 (rows are independent):
+    numpy float64 matmul of the dequantized operands."""
+    N, K = 256, 384
+    a, sa, b, sb = _case(mode, M, N, K, seed=900 + M + mode)
+    y, asum = oracle.gemm(mode, a, sa, b, sb, M, N, K)
+    A = _dequant_a(a, sa)
+    B = _dequant_b(mode, b, sb, N, K)
+    assert y.shape == (M, N)
+    assert np.all(np.abs(y - A @ B.T) <= 1e-12 * (np.abs(A) @ np.abs(B).T) + 1e-300)
+
+
+@pytest.mark.parametrize("K", [16, 200, 400])
+def test_gemm_ragged_reduction_wgrad(K):
+    """WGRAD over K tokens not a multiple of 128: the last reduction block holds
+    K mod 128 tokens and carries its own (partial-group) scales."""
+    M, N = 128, 256
+    rng = np.random.default_rng(K)
+    KB = (K + 127) // 128
+    a = _rand_codes(rng, (M, K)); sa = _rand_scales(rng, (KB, M))
+    b = _rand_codes(rng, (N, K)); sb = _rand_scales(rng, (KB, N))
+    y, asum = oracle.gemm(oracle.WGRAD, a, sa, b, sb, M, N, K)
+    A = _dequant_a_ragged(a, sa, K)
+    B = VALS[b] * np.repeat(sb.astype(np.float64), 128, axis=0)[:K].T
+    assert np.all(np.abs(y - A @ B.T) <= 1e-12 * (np.abs(A) @ np.abs(B).T) + 1e-300)
+    assert np.allclose(asum, np.abs(A) @ np.abs(B).T, rtol=1e-12, atol=0)
+
+
+def test_gemm_ragged_wgrad_through_the_layer():
+    """The layer's wgrad over 200 tokens, from the oracle's own token-wise quantizer,
+    equals the same computation on the inputs zero-padded to 256 tokens."""
+    T, Din, Dout = 200, 256, 128
+    X = synth.normal_bf16(T, Din, 1.0, seed=synth.seed_for(200, 0), outliers=True)
+    dY = synth.normal_bf16(T, Dout, 1e-3, seed=synth.seed_for(200, 2))
+    a, sa = oracle.quant_act_t(dY)
+    b, sb = oracle.quant_act_t(X)
+    y, _ = oracle.gemm(oracle.WGRAD, a, sa, b, sb, Dout, Din, T)
+    pad = lambda v: np.concatenate([v, np.zeros((256 - T, v.shape[1]), dtype=np.uint16)])
+    ap, sap = oracle.quant_act_t(pad(dY))
+    bp, sbp = oracle.quant_act_t(pad(X))
+    yp, _ = oracle.gemm(oracle.WGRAD, ap, sap, bp, sbp, Dout, Din, 256)
+    assert np.array_equal(y, yp)
+
+
+def test_gemm_ragged_bad_sizes():
+    rng = np.random.default_rng(1)
+    a = _rand_codes(rng, (128, 200)); sa = _rand_scales(rng, (2, 128))
+    b = _rand_codes(rng, (128, 200)); sb = _rand_scales(rng, (2, 128))
+    with pytest.raises(ValueError):   # FPROP reduction = features: whole blocks only
+        oracle.gemm(oracle.FPROP, a, sa, b, sb, 128, 128, 200)

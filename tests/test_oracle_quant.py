@@ -153,6 +153,54 @@ def test_weight_layout_and_transpose():
 
 def test_bad_sizes_rejected():
     with pytest.raises(ValueError):
-        oracle.quant_act(np.zeros((100, 128), dtype=np.uint16))
+        oracle.quant_act(np.zeros((128, 200), dtype=np.uint16))   # features not a multiple of 128
+    with pytest.raises(ValueError):
+        oracle.quant_act_t(np.zeros((100, 64), dtype=np.uint16))
     with pytest.raises(ValueError):
         oracle.quant_weight(np.zeros((128, 200), dtype=np.uint16))
+    with pytest.raises(ValueError):
+        oracle.quant_weight(np.zeros((100, 128), dtype=np.uint16))  # weights stay whole blocks
+
+
+# ---- token counts that are not a multiple of 128 (the last token group is partial) ----
+
+def test_act_t_partial_group_exact():
+    """M = 147 tokens: per column, one full group of 128 and a last group of the 19
+    tokens present; every group's codes and scale against the exact rational
+    checker run on exactly those values (the scale is amax/448 over the 19 present
+    tokens, not over a padded 128)."""
+    M, K = 147, 128
+    x = synth.normal_bf16(M, K, 1.0, seed=synth.seed_for(147, 0), outliers=True)
+    qt, st = oracle.quant_act_t(x)
+    assert qt.shape == (K, M) and st.shape == (2, K)
+    for k in range(0, K, 7):
+        for mb, (r0, r1) in enumerate(((0, 128), (128, M))):
+            codes, sc = quantize_group_exact(x[r0:r1, k])
+            assert list(qt[k, r0:r1]) == codes, (k, mb)
+            assert np.float32(st[mb, k]) == np.float32(float(sc)), (k, mb)
+
+
+def test_act_t_ragged_equals_zero_padded():
+    """Zero tokens change no amax, so the ragged result equals the quantization of the
+    input zero-padded to a multiple of 128 tokens, restricted to the tokens present."""
+    for M in (16, 200, 272):
+        K = 256
+        x = synth.normal_bf16(M, K, 1.0, seed=synth.seed_for(M, 1), outliers=True)
+        pad = np.zeros(((M + 127) // 128 * 128, K), dtype=np.uint16)
+        pad[:M] = x
+        qt, st = oracle.quant_act_t(x)
+        qtp, stp = oracle.quant_act_t(pad)
+        assert np.array_equal(qt, qtp[:, :M])
+        assert np.array_equal(st.view(np.uint32), stp.view(np.uint32))
+
+
+def test_act_ragged_rows_independent():
+    """Groups along K: each token row is quantized on its own, so M = 37 rows equal
+    the first 37 rows of a 128-row call on the same values."""
+    K = 384
+    big = synth.normal_bf16(128, K, 1.0, seed=synth.seed_for(37, 2), outliers=True)
+    q, s = oracle.quant_act(big[:37])
+    qb, sb = oracle.quant_act(big)
+    assert q.shape == (37, K) and s.shape == (K // 128, 37)
+    assert np.array_equal(q, qb[:37])
+    assert np.array_equal(s.view(np.uint32), sb[:, :37].view(np.uint32))
