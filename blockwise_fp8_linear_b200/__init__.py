@@ -147,13 +147,31 @@ def _on(device):
     return torch.cuda.device(device)
 
 
-def _x2(x, name):
+def _tokens(M):
+    """A token count (the M of the activation quantizers and of FPROP/DGRAD, the
+    reduction K of WGRAD) may end in a partial group of 128: a positive multiple of
+    16 (the 16-byte row stride of the token-major codes)."""
+    if int(M) <= 0 or int(M) % 16:
+        raise ValueError(f"token count {M} is not a positive multiple of 16")
+
+
+def _x2(x, name, tokens=False):
+    """Rows and columns of a 2-D input; with tokens=True the rows are a token count
+    (a multiple of 16), else both are multiples of 128."""
     import torch
     if not isinstance(x, torch.Tensor) or x.dim() != 2:
         raise ValueError(f"{name} must be a 2-D tensor")
     M, K = x.shape
-    _dims(M, K)
+    if tokens:
+        _tokens(M)
+        _dims(K)
+    else:
+        _dims(M, K)
     return int(M), int(K)
+
+
+def _groups(M):
+    return (int(M) + 127) // 128
 
 
 def fp8bw_last_device_error(stream=None) -> int:
@@ -168,9 +186,10 @@ def fp8bw_selftest_wait_timeout(limit_us: int, stream=None) -> None:
 
 
 def fp8_quant_act(x, q=None, s=None, stream=None):
-    """X[M][K] bf16 -> (Q[M][K] uint8 E4M3 codes, S[K/128][M] float32)."""
+    """X[M][K] bf16 -> (Q[M][K] uint8 E4M3 codes, S[K/128][M] float32); M any
+    multiple of 16 tokens."""
     import torch
-    M, K = _x2(x, "x")
+    M, K = _x2(x, "x", tokens=True)
     dev = _validate([(x, torch.bfloat16, (M, K), "x"), (q, torch.uint8, (M, K), "q"),
                      (s, torch.float32, (K // 128, M), "s")])
     q = _alloc(q, (M, K), torch.uint8, dev)
@@ -182,13 +201,14 @@ def fp8_quant_act(x, q=None, s=None, stream=None):
 
 
 def fp8_quant_act_t(x, qt=None, st=None, stream=None):
-    """X[M][K] bf16 -> (Q^T[K][M] uint8, S^T[M/128][K] float32), groups along M."""
+    """X[M][K] bf16 -> (Q^T[K][M] uint8, S^T[ceil(M/128)][K] float32), groups along M
+    (the last group holds the M mod 128 tokens present)."""
     import torch
-    M, K = _x2(x, "x")
+    M, K = _x2(x, "x", tokens=True)
     dev = _validate([(x, torch.bfloat16, (M, K), "x"), (qt, torch.uint8, (K, M), "qt"),
-                     (st, torch.float32, (M // 128, K), "st")])
+                     (st, torch.float32, (_groups(M), K), "st")])
     qt = _alloc(qt, (K, M), torch.uint8, dev)
-    st = _alloc(st, (M // 128, K), torch.float32, dev)
+    st = _alloc(st, (_groups(M), K), torch.float32, dev)
     with _on(dev):
         _check(lib().fp8_quant_act_t(x.data_ptr(), M, K, qt.data_ptr(), st.data_ptr(),
                                      _stream(stream)), "fp8_quant_act_t")
@@ -198,14 +218,14 @@ def fp8_quant_act_t(x, qt=None, st=None, stream=None):
 def fp8_quant_act_dual(x, q=None, s=None, qt=None, st=None, stream=None):
     """X[M][K] bf16 -> (Q, S, Q^T, S^T): both layouts from one read of X."""
     import torch
-    M, K = _x2(x, "x")
+    M, K = _x2(x, "x", tokens=True)
     dev = _validate([(x, torch.bfloat16, (M, K), "x"), (q, torch.uint8, (M, K), "q"),
                      (s, torch.float32, (K // 128, M), "s"), (qt, torch.uint8, (K, M), "qt"),
-                     (st, torch.float32, (M // 128, K), "st")])
+                     (st, torch.float32, (_groups(M), K), "st")])
     q = _alloc(q, (M, K), torch.uint8, dev)
     s = _alloc(s, (K // 128, M), torch.float32, dev)
     qt = _alloc(qt, (K, M), torch.uint8, dev)
-    st = _alloc(st, (M // 128, K), torch.float32, dev)
+    st = _alloc(st, (_groups(M), K), torch.float32, dev)
     with _on(dev):
         _check(lib().fp8_quant_act_dual(x.data_ptr(), M, K, q.data_ptr(), s.data_ptr(),
                                         qt.data_ptr(), st.data_ptr(), _stream(stream)),
@@ -235,12 +255,19 @@ def _gemm_shapes(mode: int, M: int, N: int, K: int, e8m0: bool = False):
     """Operand shapes of each GEMM mode (include/fp8bw.h): a, sa, b, sb."""
     if mode not in (FPROP, DGRAD, WGRAD):
         raise ValueError(f"mode must be FPROP, DGRAD or WGRAD, got {mode}")
-    _dims(M, N, K)
+    if e8m0:
+        _dims(M, N, K)
+    elif mode == WGRAD:   # the reduction runs over tokens
+        _dims(M, N)
+        _tokens(K)
+    else:                 # M is the token count
+        _tokens(M)
+        _dims(N, K)
     a = (M, K)
     b = (K, N) if mode == DGRAD else (N, K)
     if not e8m0:
-        sa = (K // 128, M)
-        sb = {FPROP: (N // 128, K // 128), DGRAD: (K // 128, N // 128), WGRAD: (K // 128, N)}[mode]
+        sa = (_groups(K), M)
+        sb = {FPROP: (N // 128, K // 128), DGRAD: (K // 128, N // 128), WGRAD: (_groups(K), N)}[mode]
     else:  # 512-byte scale blocks, one per 128 rows x 128-deep reduction block
         sa = (M // 128, (K // 128) * 512)
         sb = (K // 128, (N // 128) * 512) if mode == DGRAD else (N // 128, (K // 128) * 512)

@@ -79,6 +79,14 @@ bool dim_ok(int64_t d)
     return d > 0 && d <= FP8BW_MAX_DIM && (d % 128) == 0;
 }
 
+// A token count: the M of the activation quantizers and of FPROP/DGRAD, the
+// reduction K of WGRAD.  Its last group of 128 may be partial; it must be a multiple
+// of 16, the 16-byte row stride of the token-major codes and TMA's coordinate rule.
+bool tok_ok(int64_t d)
+{
+    return d > 0 && d <= FP8BW_MAX_DIM && (d % 16) == 0;
+}
+
 int from_cuda(cudaError_t e)
 {
     return e == cudaSuccess ? FP8BW_OK : FP8BW_ECUDA;
@@ -92,7 +100,7 @@ int fp8_quant_act(const void *x_bf16, int64_t M, int64_t K, uint8_t *q, float *s
 {
     if (!x_bf16 || !q || !s)
         return FP8BW_EINVAL;
-    if (!dim_ok(M) || !dim_ok(K))
+    if (!tok_ok(M) || !dim_ok(K))
         return FP8BW_ESHAPE;
     if (!aligned16(x_bf16) || !aligned16(q) || !aligned16(s))
         return FP8BW_EALIGN;
@@ -109,7 +117,7 @@ int fp8_quant_act_t(const void *x_bf16, int64_t M, int64_t K, uint8_t *qt, float
 {
     if (!x_bf16 || !qt || !st_)
         return FP8BW_EINVAL;
-    if (!dim_ok(M) || !dim_ok(K))
+    if (!tok_ok(M) || !dim_ok(K))
         return FP8BW_ESHAPE;
     if (!aligned16(x_bf16) || !aligned16(qt) || !aligned16(st_))
         return FP8BW_EALIGN;
@@ -125,7 +133,7 @@ int fp8_quant_act_dual(const void *x_bf16, int64_t M, int64_t K, uint8_t *q, flo
 {
     if (!x_bf16 || !q || !s || !qt || !st_)
         return FP8BW_EINVAL;
-    if (!dim_ok(M) || !dim_ok(K))
+    if (!tok_ok(M) || !dim_ok(K))
         return FP8BW_ESHAPE;
     if (!aligned16(x_bf16) || !aligned16(q) || !aligned16(s) || !aligned16(qt) || !aligned16(st_))
         return FP8BW_EALIGN;
@@ -227,7 +235,8 @@ int fp8_gemm_blockwise(int mode, const uint8_t *a, const float *sa, const uint8_
 {
     if (mode < FP8BW_FPROP || mode > FP8BW_WGRAD || !a || !sa || !b || !sb || !d_bf16)
         return FP8BW_EINVAL;
-    if (!dim_ok(M) || !dim_ok(N) || !dim_ok(K))
+    // the token count is M for FPROP/DGRAD and the reduction K for WGRAD
+    if (!dim_ok(N) || (mode == FP8BW_WGRAD ? !dim_ok(M) || !tok_ok(K) : !tok_ok(M) || !dim_ok(K)))
         return FP8BW_ESHAPE;
     if (!aligned16(a) || !aligned16(sa) || !aligned16(b) || !aligned16(sb) || !aligned16(d_bf16))
         return FP8BW_EALIGN;
@@ -244,7 +253,7 @@ int fp8_gemm_wgrad_acc32(const uint8_t *a, const float *sa, const uint8_t *b, co
 {
     if (!a || !sa || !b || !sb || !dw32)
         return FP8BW_EINVAL;
-    if (!dim_ok(M) || !dim_ok(N) || !dim_ok(K))
+    if (!dim_ok(M) || !dim_ok(N) || !tok_ok(K))  // K: tokens
         return FP8BW_ESHAPE;
     if (!aligned16(a) || !aligned16(sa) || !aligned16(b) || !aligned16(sb) || !aligned16(dw32))
         return FP8BW_EALIGN;
@@ -262,7 +271,8 @@ const char *fp8bw_status_string(int status)
     case FP8BW_OK: return "FP8BW_OK";
     case FP8BW_EINVAL: return "FP8BW_EINVAL: null pointer or invalid mode";
     case FP8BW_EALIGN: return "FP8BW_EALIGN: pointer not 16-byte aligned";
-    case FP8BW_ESHAPE: return "FP8BW_ESHAPE: size not a positive multiple of 128 (or too large)";
+    case FP8BW_ESHAPE:
+        return "FP8BW_ESHAPE: size not a positive multiple of 128 (16 for a token count), or too large";
     case FP8BW_ECUDA: return "FP8BW_ECUDA: CUDA runtime error";
     case FP8BW_ETIMEOUT: return "FP8BW_ETIMEOUT: a bounded in-kernel wait ran out";
     case FP8BW_EUNSUPPORTED: return "FP8BW_EUNSUPPORTED: device is not sm_100";

@@ -160,9 +160,12 @@ fp8_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__
     const int rank = (CG == 2) ? int(cluster_ctarank()) : 0;
     const int unit = (CG == 2) ? int(cluster_id_x()) : int(blockIdx.x);      // tile walker
     const int units = (CG == 2) ? int(cluster_count_x()) : int(gridDim.x);
-    const int tiles_m = M / Cfg::TILE_M, tiles_n = N / BN;
+    // A token count that is not a multiple of 128 (M for FPROP/DGRAD, K for WGRAD)
+    // ends in a partial tile / reduction block: TMA reads zeros past the end of A and
+    // B and clips the stores; the scale loader and the direct stores guard the rest.
+    const int tiles_m = (M + Cfg::TILE_M - 1) / Cfg::TILE_M, tiles_n = N / BN;
     const int num_tiles = tiles_m * tiles_n;
-    const int KB = K / BK;
+    const int KB = (K + BK - 1) / BK;
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < STAGES; ++s) {
@@ -322,7 +325,14 @@ fp8_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__
                     if (!__all_sync(0xffffffffu, ok))
                         goto role_done;
                     float *slot = sring + r * Cfg::SLOT_FLOATS;
-                    cp_async_16(slot + 4 * lane, sa_tile + size_t(kb) * M + 4 * lane);
+                    if (MODE == 2) {  // the CTA's 128 row scales (M is a feature count)
+                        cp_async_16(slot + 4 * lane, sa_tile + size_t(kb) * M + 4 * lane);
+                    } else {  // M counts tokens: rows past M (a partial tile) read as zeros
+                        const int row = tm * Cfg::TILE_M + rank * BM + 4 * lane;
+                        cp_async_16_zfill(slot + 4 * lane,
+                                          row < M ? sa_tile + size_t(kb) * M + 4 * lane : sa,
+                                          row < M);
+                    }
                     if (MODE == 0) {
                         if (lane < BN / 128)
                             cp_async_4(slot + BM + lane, sb + size_t(nb0 + lane) * KB + kb);
@@ -596,18 +606,20 @@ fp8_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__
                 } else {
                     __nv_bfloat16 *dst = D + size_t(tm * Cfg::TILE_M + row_in_tile) * size_t(N) +
                                          size_t(tn * BN + col0);
+                    if (tm * Cfg::TILE_M + row_in_tile < M) {  // rows past M: not stored
 #pragma unroll
-                    for (int c = 0; c < COLS / 8; ++c) {
-                        uint4 o;
-                        __nv_bfloat162 h0 = __float22bfloat162_rn(acc[4 * c + 0]);
-                        __nv_bfloat162 h1 = __float22bfloat162_rn(acc[4 * c + 1]);
-                        __nv_bfloat162 h2 = __float22bfloat162_rn(acc[4 * c + 2]);
-                        __nv_bfloat162 h3 = __float22bfloat162_rn(acc[4 * c + 3]);
-                        o.x = *reinterpret_cast<uint32_t *>(&h0);
-                        o.y = *reinterpret_cast<uint32_t *>(&h1);
-                        o.z = *reinterpret_cast<uint32_t *>(&h2);
-                        o.w = *reinterpret_cast<uint32_t *>(&h3);
-                        *reinterpret_cast<uint4 *>(dst + c * 8) = o;
+                        for (int c = 0; c < COLS / 8; ++c) {
+                            uint4 o;
+                            __nv_bfloat162 h0 = __float22bfloat162_rn(acc[4 * c + 0]);
+                            __nv_bfloat162 h1 = __float22bfloat162_rn(acc[4 * c + 1]);
+                            __nv_bfloat162 h2 = __float22bfloat162_rn(acc[4 * c + 2]);
+                            __nv_bfloat162 h3 = __float22bfloat162_rn(acc[4 * c + 3]);
+                            o.x = *reinterpret_cast<uint32_t *>(&h0);
+                            o.y = *reinterpret_cast<uint32_t *>(&h1);
+                            o.z = *reinterpret_cast<uint32_t *>(&h2);
+                            o.w = *reinterpret_cast<uint32_t *>(&h3);
+                            *reinterpret_cast<uint4 *>(dst + c * 8) = o;
+                        }
                     }
                 }
 #pragma unroll
@@ -783,7 +795,7 @@ static cudaError_t run(const uint8_t *a, const float *sa, const uint8_t *b, cons
         return cudaErrorInvalidValue;
     if (Cfg::TMA_STORE && Cfg::OUT32 && !make_map_f32_out(&td, d, uint64_t(M), uint64_t(N)))
         return cudaErrorInvalidValue;
-    const int64_t tiles = (M / Cfg::TILE_M) * (N / Cfg::BN);
+    const int64_t tiles = ((M + Cfg::TILE_M - 1) / Cfg::TILE_M) * (N / Cfg::BN);
     void *dp = d;
     cudaLaunchConfig_t cfg = {};
     cudaLaunchAttribute at[2];
@@ -826,7 +838,7 @@ cudaError_t launch_gemm(int mode, const uint8_t *a, const float *sa, const uint8
     // Single-CTA path: 128-wide tiles when N is not a multiple of 256, and also when
     // 256-wide ones would leave most SMs idle (fewer tiles than half the SMs, e.g. the
     // 128 x 1024 x 1024 single-layer fprop: 4 tiles of 128 x 256 or 8 of 128 x 128).
-    const bool wide = (N % 256) == 0 && (M / 128) * (N / 256) * 2 >= num_sms;
+    const bool wide = (N % 256) == 0 && ((M + 127) / 128) * (N / 256) * 2 >= num_sms;
     const bool pair = FP8BW_PAIR && (N % PBN) == 0 && (M % 256) == 0 &&
                       (M / 256) * (N / PBN) >= 16;
     switch (mode) {

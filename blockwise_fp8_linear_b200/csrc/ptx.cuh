@@ -260,6 +260,15 @@ __device__ __forceinline__ void cp_async_16(void *dst, const void *src)
                  : "memory");
 }
 
+// 16-byte cp.async that reads nothing and writes zeros when `valid` is false (src-size
+// 0); `src` must still be a valid address.
+__device__ __forceinline__ void cp_async_16_zfill(void *dst, const void *src, bool valid)
+{
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(smem_u32(dst)), "l"(src),
+                 "r"(valid ? 16u : 0u)
+                 : "memory");
+}
+
 // Arrive on `bar` once every cp.async this thread issued so far has landed (the
 // arrival counts toward the barrier's expected count).
 __device__ __forceinline__ void cp_async_mbar_arrive(uint64_t *bar)

@@ -344,7 +344,7 @@ quant_tile_kernel(const __grid_constant__ CUtensorMap tmX, int64_t M, int64_t K,
         if constexpr (E8) {
             const int e = e8m0_exponent(amax);
             g0 = amax != 0.0f ? pow2_neg(e) : 0.0f;
-            if ((sub & 1) == 0)
+            if ((sub & 1) == 0 && m_own < M)
                 *reinterpret_cast<uint32_t *>(static_cast<uint8_t *>(s_out) +
                                               ((m_own >> 7) * (K / 128) + kb) * 512 +
                                               sf_block_off(int(m_own & 127))) = rep4_code(e, amax);
@@ -352,7 +352,7 @@ quant_tile_kernel(const __grid_constant__ CUtensorMap tmX, int64_t M, int64_t K,
             g0 = __fdiv_rn(amax, 448.0f);
             const GroupDiv d(g0);
             g1 = d.fast ? d.r : -1.0f;
-            if ((sub & 1) == 0)
+            if ((sub & 1) == 0 && m_own < M)
                 static_cast<float *>(s_out)[kb * M + m_own] = g0;
         }
 #pragma unroll
@@ -369,7 +369,8 @@ quant_tile_kernel(const __grid_constant__ CUtensorMap tmX, int64_t M, int64_t K,
                 if (gp != 0.0f)
                     codes = rp > 0.0f ? quant8_fast(v, rp, gp) : quant8_ieee(v, gp);
             }
-            q[(m * K + kb * 128) / 8 + sub] = codes;
+            if (m < M)  // rows past M (a partial last tile) read as zeros and are not stored
+                q[(m * K + kb * 128) / 8 + sub] = codes;
         }
     }
     if (COLS) {
@@ -440,10 +441,16 @@ quant_tile_kernel(const __grid_constant__ CUtensorMap tmX, int64_t M, int64_t K,
         const int64_t m0 = mb * 128 + rq * 32;
         uint4 *dlo_p = reinterpret_cast<uint4 *>(qt + c * M + m0);
         uint4 *dhi_p = reinterpret_cast<uint4 *>(qt + (c + 1) * M + m0);
-        dlo_p[0] = make_uint4(clo[0], clo[1], clo[2], clo[3]);
-        dlo_p[1] = make_uint4(clo[4], clo[5], clo[6], clo[7]);
-        dhi_p[0] = make_uint4(chi[0], chi[1], chi[2], chi[3]);
-        dhi_p[1] = make_uint4(chi[4], chi[5], chi[6], chi[7]);
+        // A partial last token group (M a multiple of 16): rows past M read as zeros
+        // (no effect on the amax) and their 16-byte pieces of qt are not stored.
+        if (m0 < M) {
+            dlo_p[0] = make_uint4(clo[0], clo[1], clo[2], clo[3]);
+            dhi_p[0] = make_uint4(chi[0], chi[1], chi[2], chi[3]);
+        }
+        if (m0 + 16 < M) {
+            dlo_p[1] = make_uint4(clo[4], clo[5], clo[6], clo[7]);
+            dhi_p[1] = make_uint4(chi[4], chi[5], chi[6], chi[7]);
+        }
         if (rq == 0) {
             if (E8) {
                 uint8_t *blk = static_cast<uint8_t *>(st_out) + ((c >> 7) * (M / 128) + mb) * 512;
@@ -494,7 +501,7 @@ static cudaError_t run_tile(const void *x, int64_t M, int64_t K, void *q, void *
     cudaLaunchConfig_t cfg = {};
     cudaLaunchAttribute at[1];
     set_pdl(at[0]);
-    cfg.gridDim = dim3(unsigned(K / 128), unsigned(M / 128));
+    cfg.gridDim = dim3(unsigned(K / 128), unsigned((M + 127) / 128));  // last tile may be partial
     cfg.blockDim = dim3(QD_THREADS);
     cfg.stream = stream;
     cfg.attrs = at;

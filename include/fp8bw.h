@@ -25,7 +25,16 @@
  *                1x128 scale tensors are reduction-block-major, s[kb][row], so one
  *                tile's scales for one reduction block are contiguous.
  *   Sizes        Every dimension must be a positive multiple of 128 and at most
- *                FP8BW_MAX_DIM (else FP8BW_ESHAPE).
+ *                FP8BW_MAX_DIM (else FP8BW_ESHAPE), except a token count: the M of
+ *                fp8_quant_act, fp8_quant_act_t, fp8_quant_act_dual and of the FPROP
+ *                and DGRAD GEMMs, and the reduction K of the WGRAD GEMM and of
+ *                fp8_gemm_wgrad_acc32, which need only be a positive multiple of 16
+ *                (the 16-byte row stride of token-major codes).  The last group of
+ *                128 tokens may then be partial: its amax and scale are taken over
+ *                the tokens present (the result of zero-padding the tokens to a
+ *                multiple of 128, restricted to the tokens present), so token-wise
+ *                scale arrays have ceil(tokens/128) rows.  The E8M0 entry points
+ *                keep whole groups.
  *   Alignment    Every pointer must be 16-byte aligned (else FP8BW_EALIGN).
  *   Streams      `stream` is a cudaStream_t (NULL = legacy default stream).  Work is
  *                enqueued asynchronously; no call synchronizes the stream.  Calls on
@@ -53,7 +62,7 @@ typedef enum {
     FP8BW_OK = 0,
     FP8BW_EINVAL = 1,      /* null pointer or bad mode */
     FP8BW_EALIGN = 2,      /* a pointer is not 16-byte aligned */
-    FP8BW_ESHAPE = 3,      /* a size is not a positive multiple of 128, or too large */
+    FP8BW_ESHAPE = 3,      /* a size is not a positive multiple of 128 (16 for a token count), or too large */
     FP8BW_ECUDA = 4,       /* a CUDA runtime call or kernel launch failed */
     FP8BW_ETIMEOUT = 5,    /* a bounded in-kernel wait ran out (from fp8bw_last_device_error) */
     FP8BW_EUNSUPPORTED = 6 /* the current device is not sm_100 */
@@ -80,7 +89,7 @@ int fp8_quant_act(const void *x_bf16, int64_t M, int64_t K, uint8_t *q, float *s
  * fp8_quant_act_t -- the same groups taken along M (the token dimension), the
  * grouping wgrad needs because its reduction runs over tokens (section 3.2: wgrad
  * runs in FP8 on the layer's inputs and output gradients).
- *   x  [M][K] BF16 in      qt [K][M] E4M3 codes out (transposed)      st [M/128][K] FP32 out
+ *   x  [M][K] BF16 in      qt [K][M] E4M3 codes out (transposed)      st [ceil(M/128)][K] FP32 out
  * For each column k and block mb: the group is x[mb*128 .. mb*128+127][k];
  * st[mb][k] is its scale and qt[k][mb*128 + i] its codes.  Quantized from the BF16
  * tensor, not from the row-wise FP8 copy.
@@ -96,7 +105,7 @@ int fp8_quant_act_t(const void *x_bf16, int64_t M, int64_t K, uint8_t *qt, float
  * fp8_quant_act_t(x, M, K, qt, st):
  *   x [M][K] BF16 in
  *   q [M][K], s [K/128][M]      1x128 groups along K
- *   qt [K][M], st [M/128][K]    1x128 groups along M (codes transposed)
+ *   qt [K][M], st [ceil(M/128)][K]    1x128 groups along M (codes transposed)
  */
 int fp8_quant_act_dual(const void *x_bf16, int64_t M, int64_t K, uint8_t *q, float *s,
                        uint8_t *qt, float *st, void *stream);
@@ -128,7 +137,9 @@ int fp8_quant_weight(const void *w_bf16, int64_t N, int64_t K, uint8_t *q, float
  *                         fp8_quant_weight produced it, [out][in]; read transposed)
  *                         M = tokens, K = out_features, N = in_features
  *   WGRAD  dW = dY^T . X  a = Qdy^T [M][K], sa = [K/128][M] (from fp8_quant_act_t(dY))
- *                         b = Qx^T  [N][K], sb = [K/128][N] (from fp8_quant_act_t(X))
+ *                         b = Qx^T  [N][K], sb = [K/128][N] (from fp8_quant_act_t(X));
+ *                         with K tokens not a multiple of 128, sa and sb have
+ *                         ceil(K/128) rows, the last for the partial token group
  *                         M = out_features, K = tokens, N = in_features
  * d_bf16 [M][N] is written, never read.
  */
