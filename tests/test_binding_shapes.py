@@ -97,3 +97,30 @@ def test_wgrad_acc32_checks_the_fp32_buffer():
 def test_bad_mode_is_rejected():
     with pytest.raises(ValueError):
         fb.fp8_gemm_blockwise(3, *gemm_args(fb.FPROP), M, N, K)
+
+
+# ---- token counts that are not a multiple of 128 ----
+
+def test_ragged_token_shapes():
+    """A token count only needs to be a multiple of 16; token-wise scale arrays then
+    have ceil(tokens/128) rows, and the feature dimensions stay multiples of 128."""
+    T = 144
+    assert fb._gemm_shapes(fb.FPROP, T, N, K) == ((T, K), (K // 128, T), (N, K), (N // 128, K // 128))
+    assert fb._gemm_shapes(fb.WGRAD, M, N, T) == ((M, T), (2, M), (N, T), (2, N))
+    with pytest.raises(ValueError):
+        fb._gemm_shapes(fb.FPROP, 136, N, K)          # not a multiple of 16
+    with pytest.raises(ValueError):
+        fb._gemm_shapes(fb.FPROP, T, N, 144)          # FPROP reduction = features
+    with pytest.raises(ValueError):
+        fb._gemm_shapes(fb.WGRAD, 144, N, T)          # WGRAD M = features
+    with pytest.raises(ValueError):
+        fb._gemm_shapes(fb.FPROP, T, N, K, True)      # E8M0 keeps whole groups
+    xr = z(T, 384, dtype=bf16)
+    with pytest.raises(ValueError):   # st must have ceil(144/128) = 2 rows
+        fb.fp8_quant_act_t(xr, st=z(1, 384, dtype=f32))
+    with pytest.raises(ValueError):
+        fb.fp8_quant_act_dual(xr, st=z(1, 384, dtype=f32))
+    with pytest.raises(TypeError):    # the right shapes pass and stop at the device check
+        fb.fp8_quant_act_t(xr, qt=z(384, T), st=z(2, 384, dtype=f32))
+    with pytest.raises(ValueError):   # weights stay whole blocks
+        fb.fp8_quant_weight(xr)
