@@ -558,13 +558,17 @@ def run_ours(args):
         torch.cuda.synchronize()
         t0 = torch.cuda.Event(enable_timing=True)
         t1 = torch.cuda.Event(enable_timing=True)
+        marks = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
         t0.record()
-        for _ in range(args.steps):
+        for i in range(args.steps):
             work.step(side=side, reducer=reducer)
+            marks[i].record()  # end of step i on the main stream (it waits for the side one)
         t1.record()
         torch.cuda.synchronize()
         barrier(world)
     local_ms = t0.elapsed_time(t1)
+    step_ms = [t0.elapsed_time(marks[0])] + [marks[i - 1].elapsed_time(marks[i])
+                                             for i in range(1, args.steps)]
     elapsed_ms = max_over_ranks(local_ms, world)
     if fb.fp8bw_last_device_error() != 0:
         raise RuntimeError("a bounded in-kernel wait ran out in the timed region")
@@ -572,6 +576,10 @@ def run_ours(args):
 
     ms_per_step = elapsed_ms / args.steps
     value = world * STEP_FLOPS / (ms_per_step * 1e-3) / 1e12
+    pct = np.percentile(np.array(step_ms), [10, 50, 90])
+    step_percentiles = {"p10": round(float(pct[0]), 4), "p50": round(float(pct[1]), 4),
+                        "p90": round(float(pct[2]), 4), "unit": "ms",
+                        "of": "per-step device time of the timed steps (rank 0)"}
 
     # sustained: the same step repeated for a few seconds, deep into the power cap
     sustained = None
@@ -757,6 +765,7 @@ def run_ours(args):
                                   dp_grad=reducer is not None), "roofline": roofline,
             "cpu_baseline": cpu,
             "e2e": e2e, "gpu_launches": work.launches_per_step * args.steps,
+            "step_ms_percentiles": step_percentiles,
             "clocks": clock_info,
             "pct_of_fp8_peak": round(100 * value / world / fp8_peak, 2),
             "pct_of_nominal_fp8_peak": round(100 * value / world / NOMINAL_FP8_TFLOPS, 2),
@@ -773,16 +782,18 @@ def run_ours(args):
 
 # ----------------------------------------------------- oracle (CPU) timing
 
-def oracle_sample_step(i, host, threads):
+def oracle_sample_step(i, host, threads, tokens=TOKENS):
     """One bounded sample of the step on the CPU oracle: linear i % 4, GEMM mode
     (i // 4) % 3, one 128-row tile of the output, with the quantization of exactly
-    the groups that tile reads.  Returns (GEMM flops done, seconds)."""
+    the groups that tile reads; `tokens` of the host inputs are used.  Returns (GEMM
+    flops done, seconds)."""
     import oracle
     li = i % len(LINEARS)
     mode = (i // len(LINEARS)) % 3
     name, din, dout = LINEARS[li]
     X, W, dY = host[li]
-    r0 = 128 * ((i // 12) % (TOKENS // 128))
+    X, dY = X[:tokens], dY[:tokens]
+    r0 = 128 * ((i // 12) % (tokens // 128))
     t = time.perf_counter()
     if mode == oracle.FPROP:
         a, sa = oracle.quant_act(np.ascontiguousarray(X[r0:r0 + 128]))
@@ -795,8 +806,8 @@ def oracle_sample_step(i, host, threads):
     else:
         # output rows r0..r0+127 of dW (out-features): those columns of dY, all tokens
         a, sa = oracle.quant_act_t(np.ascontiguousarray(dY[:, r0 % dout:(r0 % dout) + 128]))
-        b, sb = oracle.quant_act_t(X)
-        M, N, K = 128, din, TOKENS
+        b, sb = oracle.quant_act_t(np.ascontiguousarray(X))
+        M, N, K = 128, din, tokens
     oracle.gemm(mode, a, sa, b, sb, M, N, K, nthreads=threads)
     return 2 * M * N * K, time.perf_counter() - t
 
@@ -1075,9 +1086,34 @@ def run_sweep(args):
         if b["value"] < 1.05 * a["value"]:
             knee = a["tokens"]
             break
-    print(json.dumps({"sweep": "knee", "knee_tokens": knee,
-                      "rule": "smallest M whose doubling gains < 5% of T_lin",
-                      "values": {r["tokens"]: r["value"] for r in results}}), flush=True)
+    line = {"sweep": "knee", "knee_tokens": knee,
+            "rule": "smallest M whose doubling gains < 5% of T_lin",
+            "values": {r["tokens"]: r["value"] for r in results}}
+    if not args.no_cpu:
+        # The CPU oracle on one layer at M = 4096 (a bounded sample of 128-row output
+        # tiles of its 12 GEMMs, with the quantization each tile reads), extrapolated
+        # linearly in FLOPs to each M's 28-layer step.
+        import oracle
+        threads = oracle.max_threads()
+        host = make_inputs(0)
+        flops, secs, n = 0, 0.0, 0
+        while secs < args.cpu_budget:
+            f, t = oracle_sample_step(n, host, threads, tokens=SWEEP_TOKENS[0])
+            flops += f
+            secs += t
+            n += 1
+        rate = flops / secs
+        line["cpu_baseline"] = {
+            "value": round(rate / 1e12, 6), "unit": UNIT, "kind": "oracle", "cores": threads,
+            "cpu_model": cpu_model(), "nproc": os.cpu_count(),
+            "sample": f"one layer at M={SWEEP_TOKENS[0]}: {n} samples, each one 128-row output "
+                      f"tile of one of the 12 GEMMs plus the quantization it reads, {secs:.1f} s",
+            "extrapolated_step_s": {
+                r["tokens"]: round(SWEEP_LAYERS * sum(3 * 2 * r["tokens"] * din * dout
+                                                      for _, din, dout in LINEARS) / rate, 1)
+                for r in results},
+            "extrapolation": "linear in FLOPs (stated as such; not measured at full size)"}
+    print(json.dumps(line), flush=True)
 
 
 def main():
