@@ -754,6 +754,15 @@ def run_ours(args):
     cpu = None
     if rank == 0 and not args.no_cpu:
         cpu = cpu_baseline(budget_s=args.cpu_budget, host=host)
+    sweep = None
+    if world == 1 and not args.no_sweep:
+        # the micro-batch knee (28-layer step linear work at M = 4096 .. 32768)
+        per_m, knee_line = run_sweep(args, emit=False, cpu_budget=min(args.cpu_budget, 5.0))
+        sweep = {"knee_tokens": knee_line["knee_tokens"], "rule": knee_line["rule"],
+                 "per_m": [{k: r[k] for k in ("tokens", "value", "ms_per_step", "gemm_tflops",
+                                              "gemm_share_of_step", "clocks")} for r in per_m],
+                 "unit": UNIT, "steps_per_m": args.sweep_steps, "layers": SWEEP_LAYERS,
+                 "cpu_baseline": knee_line.get("cpu_baseline")}
 
     if rank == 0:
         line = {
@@ -766,6 +775,7 @@ def run_ours(args):
             "cpu_baseline": cpu,
             "e2e": e2e, "gpu_launches": work.launches_per_step * args.steps,
             "step_ms_percentiles": step_percentiles,
+            "micro_batch_sweep": sweep,
             "clocks": clock_info,
             "pct_of_fp8_peak": round(100 * value / world / fp8_peak, 2),
             "pct_of_nominal_fp8_peak": round(100 * value / world / NOMINAL_FP8_TFLOPS, 2),
@@ -984,14 +994,16 @@ SWEEP_TOKENS = (4096, 8192, 16384, 32768)   # micro-batch 1, 2, 4, 8 x sequence 
 SWEEP_LAYERS = 28
 
 
-def run_sweep(args):
+def run_sweep(args, emit=True, cpu_budget=None):
     """Knee sweep of one 28-layer step's linear work: per layer the four linears of the
     block in fprop + dgrad + wgrad with all quantizers (24 launches), each layer with its
     own weights, at M = 4096 ... 32768 tokens.  Prints one JSON line per M and a
     summary line naming the knee: the smallest M whose doubling gains < 5% of T_lin.
     Inputs come from torch's seeded device generator (X ~ N(0,1) with 1% outlier
     channels x20, W ~ N(0,0.02), dY ~ N(0,1e-3)); activations are shared by the
-    layers, weights are distinct per layer (2.8 GB of BF16)."""
+    layers, weights are distinct per layer (2.8 GB of BF16).  With emit=False nothing is
+    printed and the per-M lines and the knee line are returned (the default bench run
+    carries them in its own line)."""
     import torch
     import blockwise_fp8_linear_b200 as fb
     from blockwise_fp8_linear_b200 import build as fbuild
@@ -1078,7 +1090,8 @@ def run_sweep(args):
                 "launches_per_step": SWEEP_LAYERS * 24, "clocks": clocks.summary(),
                 "data": "synthetic (torch seeded device generator)"}
         results.append(line)
-        print(json.dumps(line), flush=True)
+        if emit:
+            print(json.dumps(line), flush=True)
         del bufs
         torch.cuda.empty_cache()
     knee = None
@@ -1089,7 +1102,8 @@ def run_sweep(args):
     line = {"sweep": "knee", "knee_tokens": knee,
             "rule": "smallest M whose doubling gains < 5% of T_lin",
             "values": {r["tokens"]: r["value"] for r in results}}
-    if not args.no_cpu:
+    budget = args.cpu_budget if cpu_budget is None else cpu_budget
+    if not args.no_cpu and budget > 0:
         # The CPU oracle on one layer at M = 4096 (a bounded sample of 128-row output
         # tiles of its 12 GEMMs, with the quantization each tile reads), extrapolated
         # linearly in FLOPs to each M's 28-layer step.
@@ -1097,7 +1111,7 @@ def run_sweep(args):
         threads = oracle.max_threads()
         host = make_inputs(0)
         flops, secs, n = 0, 0.0, 0
-        while secs < args.cpu_budget:
+        while secs < budget:
             f, t = oracle_sample_step(n, host, threads, tokens=SWEEP_TOKENS[0])
             flops += f
             secs += t
@@ -1113,7 +1127,9 @@ def run_sweep(args):
                                                       for _, din, dout in LINEARS) / rate, 1)
                 for r in results},
             "extrapolation": "linear in FLOPs (stated as such; not measured at full size)"}
-    print(json.dumps(line), flush=True)
+    if emit:
+        print(json.dumps(line), flush=True)
+    return results, line
 
 
 def main():
@@ -1146,6 +1162,8 @@ def main():
                     help="with --kernel-only gemm_*: the linear whose GEMM shapes to launch")
     ap.add_argument("--quant-shape", default="8192x12288",
                     help="with --kernel-only quant_*: ROWSxCOLS of the BF16 input")
+    ap.add_argument("--no-sweep", action="store_true",
+                    help="skip the micro-batch knee sweep that the default run carries")
     ap.add_argument("--sweep", action="store_true",
                     help="micro-batch knee sweep (28 layers, M = 4096..32768); one JSON line per M")
     ap.add_argument("--sweep-steps", type=int, default=3)
