@@ -134,7 +134,7 @@ template <class Cfg>
 __global__ void __launch_bounds__(Cfg::THREADS, 1)
 fp8_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                 const __grid_constant__ CUtensorMap tmD, const float *__restrict__ sa, const float *__restrict__ sb,
-                void *__restrict__ Dv, int M, int N, int K)
+                void *__restrict__ Dv, int M, int N, int K, int tiles_m, int KB)
 {
     constexpr int BN = Cfg::BN, MODE = Cfg::MODE, STAGES = Cfg::STAGES, CG = Cfg::CG;
     constexpr int COLS = Cfg::COLS, EPI_WARPS = Cfg::EPI_WARPS;
@@ -163,9 +163,9 @@ fp8_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__
     // A token count that is not a multiple of 128 (M for FPROP/DGRAD, K for WGRAD)
     // ends in a partial tile / reduction block: TMA reads zeros past the end of A and
     // B and clips the stores; the scale loader and the direct stores guard the rest.
-    const int tiles_m = (M + Cfg::TILE_M - 1) / Cfg::TILE_M, tiles_n = N / BN;
+    const int tiles_n = N / BN;  // tiles_m and KB (ceil divisions) come from the host
     const int num_tiles = tiles_m * tiles_n;
-    const int KB = (K + BK - 1) / BK;
+
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < STAGES; ++s) {
@@ -816,7 +816,8 @@ static cudaError_t run(const uint8_t *a, const float *sa, const uint8_t *b, cons
         const int64_t clusters = tiles < max_clusters ? tiles : max_clusters;
         cfg.gridDim = dim3(unsigned(2 * clusters));
     }
-    e = cudaLaunchKernelEx(&cfg, kern, ta, tb, td, sa, sb, dp, int(M), int(N), int(K));
+    e = cudaLaunchKernelEx(&cfg, kern, ta, tb, td, sa, sb, dp, int(M), int(N), int(K),
+                           int((M + Cfg::TILE_M - 1) / Cfg::TILE_M), int((K + BK - 1) / BK));
     if (e != cudaSuccess)
         return e;
     return cudaGetLastError();
