@@ -50,6 +50,21 @@ struct GroupDiv {
     }
 };
 
+// The group scale amax / 448, correctly rounded to binary32, in three operations
+// instead of a full division: q0 = RN(amax * RN(1/448)), then one correction step
+// (Markstein's, as in GroupDiv below): d = RN(amax - q0 * 448) by FMA, s = RN(q0 + d *
+// RN(1/448)).  amax is always a non-negative BF16 value widened to FP32 (32,640
+// positive finite ones and zero); the sequence equals the IEEE quotient for every one
+// of them, checked against the exact rational quotient on the host and against the
+// oracle on the GPU for every BF16 amax.
+__device__ __forceinline__ float scale_of_amax(float amax)
+{
+    constexpr float inv448 = 1.0f / 448.0f;
+    const float q0 = __fmul_rn(amax, inv448);
+    const float d = __fmaf_rn(-q0, 448.0f, amax);
+    return __fmaf_rn(d, inv448, q0);
+}
+
 __device__ __forceinline__ float bf16lo(uint32_t w) { return __uint_as_float(w << 16); }
 __device__ __forceinline__ float bf16hi(uint32_t w) { return __uint_as_float(w & 0xFFFF0000u); }
 
@@ -197,7 +212,7 @@ quant_weight_kernel(const uint4 *__restrict__ w, int64_t N, int64_t K, uint2 *__
     for (int i = 0; i < 8; ++i)
         m2 = __vmaxu2(m2, red[i]);
     const float amax = halves_max_to_float(m2);
-    const float sc = E8 ? 0.0f : __fdiv_rn(amax, 448.0f);
+    const float sc = E8 ? 0.0f : scale_of_amax(amax);
     const int e = E8 ? e8m0_exponent(amax) : 0;
     const GroupDiv div(sc);
 
@@ -271,7 +286,9 @@ constexpr int QERR_TILE_LOAD = 21;
 constexpr uint64_t QT_WAIT_NS = 1000000000ull;
 constexpr uint64_t QT_DRAIN_NS = 20000000ull;
 
-template <bool ROWS, bool COLS, bool E8 = false>
+// RAGGED: M is not a multiple of 128, so the last row tile is partial and the stores
+// past M are skipped; whole tiles run the unguarded instantiation.
+template <bool ROWS, bool COLS, bool E8, bool RAGGED>
 __global__ void __launch_bounds__(QD_THREADS, QD_MIN_BLOCKS)
 quant_tile_kernel(const __grid_constant__ CUtensorMap tmX, int64_t M, int64_t K,
                       uint2 *__restrict__ q, void *__restrict__ s_out, uint8_t *__restrict__ qt,
@@ -344,15 +361,15 @@ quant_tile_kernel(const __grid_constant__ CUtensorMap tmX, int64_t M, int64_t K,
         if constexpr (E8) {
             const int e = e8m0_exponent(amax);
             g0 = amax != 0.0f ? pow2_neg(e) : 0.0f;
-            if ((sub & 1) == 0 && m_own < M)
+            if ((sub & 1) == 0 && (!RAGGED || m_own < M))
                 *reinterpret_cast<uint32_t *>(static_cast<uint8_t *>(s_out) +
                                               ((m_own >> 7) * (K / 128) + kb) * 512 +
                                               sf_block_off(int(m_own & 127))) = rep4_code(e, amax);
         } else {
-            g0 = __fdiv_rn(amax, 448.0f);
+            g0 = scale_of_amax(amax);
             const GroupDiv d(g0);
             g1 = d.fast ? d.r : -1.0f;
-            if ((sub & 1) == 0 && m_own < M)
+            if ((sub & 1) == 0 && (!RAGGED || m_own < M))
                 static_cast<float *>(s_out)[kb * M + m_own] = g0;
         }
 #pragma unroll
@@ -369,7 +386,7 @@ quant_tile_kernel(const __grid_constant__ CUtensorMap tmX, int64_t M, int64_t K,
                 if (gp != 0.0f)
                     codes = rp > 0.0f ? quant8_fast(v, rp, gp) : quant8_ieee(v, gp);
             }
-            if (m < M)  // rows past M (a partial last tile) read as zeros and are not stored
+            if (!RAGGED || m < M)  // rows past M (a partial last tile) read as zeros: not stored
                 q[(m * K + kb * 128) / 8 + sub] = codes;
         }
     }
@@ -387,8 +404,8 @@ quant_tile_kernel(const __grid_constant__ CUtensorMap tmX, int64_t M, int64_t K,
         m2 = __vmaxu2(__vmaxu2(red[0][cp], red[1][cp]), __vmaxu2(red[2][cp], red[3][cp]));
         const float amax_lo = __uint_as_float((m2 & 0xFFFFu) << 16);
         const float amax_hi = __uint_as_float(m2 & 0xFFFF0000u);
-        const float s_lo = E8 ? 0.0f : __fdiv_rn(amax_lo, 448.0f);
-        const float s_hi = E8 ? 0.0f : __fdiv_rn(amax_hi, 448.0f);
+        const float s_lo = E8 ? 0.0f : scale_of_amax(amax_lo);
+        const float s_hi = E8 ? 0.0f : scale_of_amax(amax_hi);
         const int e_lo = E8 ? e8m0_exponent(amax_lo) : 0;
         const int e_hi = E8 ? e8m0_exponent(amax_hi) : 0;
         uint32_t clo[8], chi[8];
@@ -443,11 +460,11 @@ quant_tile_kernel(const __grid_constant__ CUtensorMap tmX, int64_t M, int64_t K,
         uint4 *dhi_p = reinterpret_cast<uint4 *>(qt + (c + 1) * M + m0);
         // A partial last token group (M a multiple of 16): rows past M read as zeros
         // (no effect on the amax) and their 16-byte pieces of qt are not stored.
-        if (m0 < M) {
+        if (!RAGGED || m0 < M) {
             dlo_p[0] = make_uint4(clo[0], clo[1], clo[2], clo[3]);
             dhi_p[0] = make_uint4(chi[0], chi[1], chi[2], chi[3]);
         }
-        if (m0 + 16 < M) {
+        if (!RAGGED || m0 + 16 < M) {
             dlo_p[1] = make_uint4(clo[4], clo[5], clo[6], clo[7]);
             dhi_p[1] = make_uint4(chi[4], chi[5], chi[6], chi[7]);
         }
@@ -506,7 +523,10 @@ static cudaError_t run_tile(const void *x, int64_t M, int64_t K, void *q, void *
     cfg.stream = stream;
     cfg.attrs = at;
     cfg.numAttrs = 1;
-    cudaError_t e = cudaLaunchKernelEx(&cfg, quant_tile_kernel<ROWS, COLS, E8>, map, M, K,
+    cudaError_t e = cudaLaunchKernelEx(&cfg,
+                                       (M % 128) ? quant_tile_kernel<ROWS, COLS, E8, true>
+                                                 : quant_tile_kernel<ROWS, COLS, E8, false>,
+                                       map, M, K,
                                        reinterpret_cast<uint2 *>(q), s, qt, st);
     return e != cudaSuccess ? e : cudaGetLastError();
 }
