@@ -455,7 +455,9 @@ def single_fprop_latency(dev, reps=200):
     seed 0) through the C ABI: fp8_quant_act(X), fp8_quant_weight(W) and the FPROP
     GEMM.  Latency-bound, so it is reported in microseconds: device time per layer
     call (events around `reps` calls back to back) and per GEMM alone, plus the host
-    time to issue one layer call."""
+    time to issue one layer call; then the same layer captured once in a CUDA graph
+    and replayed `reps` times (no host work per kernel), with a check that the
+    replayed output equals the eager one."""
     import torch
     import blockwise_fp8_linear_b200 as fb
     from blockwise_fp8_linear_b200 import synth
@@ -471,11 +473,11 @@ def single_fprop_latency(dev, reps=200):
     Y = torch.empty(T, Dout, dtype=torch.bfloat16, device=dev)
     st = torch.cuda.current_stream().cuda_stream
 
-    def layer():
-        rc = (L.fp8_quant_act(X.data_ptr(), T, Din, qx.data_ptr(), sx.data_ptr(), st)
-              or L.fp8_quant_weight(W.data_ptr(), Dout, Din, qw.data_ptr(), sw.data_ptr(), None, st)
+    def layer(s=st):
+        rc = (L.fp8_quant_act(X.data_ptr(), T, Din, qx.data_ptr(), sx.data_ptr(), s)
+              or L.fp8_quant_weight(W.data_ptr(), Dout, Din, qw.data_ptr(), sw.data_ptr(), None, s)
               or L.fp8_gemm_blockwise(0, qx.data_ptr(), sx.data_ptr(), qw.data_ptr(),
-                                      sw.data_ptr(), Y.data_ptr(), T, Dout, Din, st))
+                                      sw.data_ptr(), Y.data_ptr(), T, Dout, Din, s))
         if rc:
             raise fb.Fp8bwError(rc, "single fprop")
 
@@ -502,6 +504,42 @@ def single_fprop_latency(dev, reps=200):
         torch.cuda.synchronize()
         out[f"{name}_us"] = round(1e3 * e0.elapsed_time(e1) / reps, 2)
         out[f"{name}_host_issue_us"] = round(1e6 * (h1 - h0) / reps, 2)
+
+    # The layer captured once (warmed up on a side stream first, then captured) and
+    # replayed: the three launches cost one graph launch on the host.
+    layer()
+    torch.cuda.synchronize()
+    y_eager = Y.clone()
+    try:
+        side = torch.cuda.Stream(device=dev)
+        side.wait_stream(torch.cuda.current_stream())
+        with torch.cuda.stream(side):
+            layer(side.cuda_stream)
+        torch.cuda.current_stream().wait_stream(side)
+        torch.cuda.synchronize()
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, capture_error_mode="relaxed"):
+            layer(torch.cuda.current_stream().cuda_stream)
+        Y.zero_()
+        for _ in range(10):
+            g.replay()
+        torch.cuda.synchronize()
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        h0 = time.perf_counter()
+        e0.record()
+        for _ in range(reps):
+            g.replay()
+        e1.record()
+        h1 = time.perf_counter()
+        torch.cuda.synchronize()
+        out["layer_graph_us"] = round(1e3 * e0.elapsed_time(e1) / reps, 2)
+        out["layer_graph_host_issue_us"] = round(1e6 * (h1 - h0) / reps, 2)
+        out["graph_output_identical"] = bool(torch.equal(Y, y_eager))
+        del g
+    except Exception as exc:  # report, do not hide, a capture the runtime refused
+        out["layer_graph_us"] = None
+        out["graph_error"] = repr(exc)[:200]
     out["unit"] = "us"
     return out
 
