@@ -38,9 +38,9 @@
  *   Alignment    Every pointer must be 16-byte aligned (else FP8BW_EALIGN).
  *   Streams      `stream` is a cudaStream_t (NULL = legacy default stream).  Work is
  *                enqueued asynchronously; no call but fp8bw_last_device_error
- *                synchronizes the stream.  Calls on
- *                distinct streams may run concurrently from different threads.  A
- *                call only enqueues kernels (it allocates nothing and waits for
+ *                synchronizes the stream.  Calls on distinct streams may run
+ *                concurrently from different threads.  A call only enqueues
+ *                kernels (it allocates nothing and waits for
  *                nothing), so it may be captured into a CUDA graph once its
  *                configuration has run eagerly on the device (the first launch of a
  *                configuration sets its shared-memory limit); fp8bw_last_device_error
