@@ -17,11 +17,11 @@
 //               CTA's rows, b-scales of the tile) into a shared-memory ring with
 //               cp.async, signalling a per-slot barrier when they land.
 //   warp 3      idle (completes the first warpgroup, which gives registers away)
-//   warps 4..11 promotion + epilogue: each thread owns one TMEM lane (a row of the
-//               tile) and COLS columns.  Per block it loads the FP32 partial from
-//               TMEM 32 columns at a time, releases the buffer, and adds partial x
-//               scale into an FP32 running sum held in registers (packed f32x2
-//               FMA).  After the last block it rounds the sum to BF16 and stores it.
+//   warps 4..11 promotion + epilogue: per block each thread loads its FP32 partial
+//               from TMEM (one lane, i.e. row, and COLS columns in 64- or 32-column
+//               loads; wgrad pairs: 4 rows x 32 columns per 16x256b load), releases
+//               the buffer and adds partial x scale into an FP32 running sum in
+//               registers (packed f32x2 FMA); last, it rounds to BF16 and stores.
 // Double-buffered TMEM partials let the tensor cores run block kb+1 while the
 // epilogue promotes block kb.
 //
